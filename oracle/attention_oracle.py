@@ -1,0 +1,251 @@
+"""fp64 CPU oracle for exact (tiled) scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  It shares no code
+with the CUDA library and imports nothing from it; the product path never
+calls it.
+
+Everything here is computed in float64 from the exact bf16 input values.  The
+functions are the plain definitions, written so that they can be checked
+against the pages by eye:
+
+* Standard attention (FlashAttention V2 deep dive, section "Attention反向传播的
+  「内存泄漏」难题", the standard-forward listing; Ascend ops-transformer
+  article, section 一 "标准注意力"):  S = Q K^T * scale, P = softmax(S) row-wise,
+  O = P V.  The per-row log-sum-exp  lse_i = log sum_j exp(s_ij)  is the
+  statistic the forward hands to the backward (deep dive, section 改进3,
+  "log-sum-exp 的计算顺序").
+* Backward by recomputation (deep dive, section 改进1 "IO感知的算子调度"):
+  P is recomputed from the saved statistic instead of being stored.  The
+  gradient of the softmax is the closed form  dS = P o (dP - D),
+  D_i = sum_j P_ij dP_ij.  The listing on that page multiplies dP by
+  (P - P^2), which is only the diagonal of the softmax Jacobian; the closed
+  form is used instead (the listing's rule is kept as a negative test).
+* The blocked variant (FlashAttention glossary, sections 2.1 "分块计算", 2.2
+  "在线Softmax", 2.3 "完整算法流程"; Ascend article, section 三 "增量 Softmax"):
+  Q is cut into row blocks, K/V into column blocks, and a running max m and
+  running sum l per row are updated block by block with the final O / l
+  correction.  The glossary's listing leaves the inner loop over j implicit,
+  takes the block max over all rows at once, and rescales O by a factor that
+  is always 1; this variant follows the per-row update the prose describes.
+
+Conventions: q, do are [B, Hq, N, D]; k, v are [B, Hkv, N, D]; query head h
+reads K/V head h // (Hq // Hkv) (contiguous groups).  Causal means key j is
+visible to query i iff j <= i.  lse is the natural log of the scaled logits.
+Parity status: every function here is pinned by tests/test_oracle_pins.py
+(closed forms, invariants, hand-worked golden values, brute force, central
+finite differences and a torch autograd cross-check).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+_ROW_CHUNK = 256
+
+
+def kv_head_of(hq: int, Hq: int, Hkv: int) -> int:
+    """GQA head map: contiguous groups of Hq/Hkv query heads share a K/V head."""
+    if Hq % Hkv != 0:
+        raise ValueError("Hq must be a multiple of Hkv")
+    return hq // (Hq // Hkv)
+
+
+def _f64(x) -> np.ndarray:
+    if hasattr(x, "detach"):  # torch tensor (possibly bf16)
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def scores(q_rows: np.ndarray, k: np.ndarray, scale: float, rows: np.ndarray, causal: bool) -> np.ndarray:
+    """s_ij = scale * q_i . k_j for the given query rows; -inf where j > i (causal)."""
+    s = scale * (q_rows @ k.T)
+    if causal:
+        cols = np.arange(k.shape[0])
+        s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+    return s
+
+
+def row_lse(s: np.ndarray) -> np.ndarray:
+    """lse_i = log sum_j exp(s_ij), evaluated as m_i + log sum_j exp(s_ij - m_i)."""
+    m = s.max(axis=1)
+    return m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+
+
+def probs(s: np.ndarray, lse: np.ndarray) -> np.ndarray:
+    """p_ij = exp(s_ij - lse_i)  (row-wise softmax of the scaled logits)."""
+    return np.exp(s - lse[:, None])
+
+
+def _head_forward(qh, kh, vh, scale, causal, rows=None):
+    N = kh.shape[0]
+    rows = np.arange(qh.shape[0]) if rows is None else np.asarray(rows)
+    o = np.empty((len(rows), vh.shape[1]))
+    lse = np.empty(len(rows))
+    for c0 in range(0, len(rows), _ROW_CHUNK):
+        r = rows[c0:c0 + _ROW_CHUNK]
+        s = scores(qh[r], kh, scale, r, causal)
+        l = row_lse(s)
+        p = probs(s, l)
+        o[c0:c0 + len(r)] = p @ vh
+        lse[c0:c0 + len(r)] = l
+    assert N == kh.shape[0]
+    return o, lse
+
+
+def attention_forward(q, k, v, scale: float, causal: bool):
+    """Naive attention, every (b, h): returns (O [B,Hq,N,D], LSE [B,Hq,N]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            o[b, h], lse[b, h] = _head_forward(q[b, h], k[b, g], v[b, g], scale, causal)
+    return o, lse
+
+
+def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, h: int, rows):
+    """O and LSE of the listed query rows of head (b, h) only (same definition)."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    g = kv_head_of(h, Hq, Hkv)
+    return _head_forward(_f64(q[b, h]), _f64(k[b, g]), _f64(v[b, g]), scale, causal, rows)
+
+
+def _head_backward(qh, kh, vh, doh, scale, causal, dk_acc, dv_acc):
+    """Closed-form gradients of L = <O, dO> for one query head.
+
+    dV_j += sum_i p_ij dO_i;  dP_ij = dO_i . v_j;  D_i = sum_j p_ij dP_ij;
+    dS_ij = p_ij (dP_ij - D_i);  dQ_i = scale sum_j dS_ij k_j;
+    dK_j += scale sum_i dS_ij q_i.
+    """
+    N = qh.shape[0]
+    dq = np.empty_like(qh)
+    for c0 in range(0, N, _ROW_CHUNK):
+        r = np.arange(c0, min(N, c0 + _ROW_CHUNK))
+        s = scores(qh[r], kh, scale, r, causal)
+        p = probs(s, row_lse(s))
+        dp = doh[r] @ vh.T
+        Di = (p * dp).sum(axis=1)
+        ds = p * (dp - Di[:, None])
+        dq[r] = scale * (ds @ kh)
+        dk_acc += scale * (ds.T @ qh[r])
+        dv_acc += p.T @ doh[r]
+    return dq
+
+
+def attention_backward(q, k, v, do, scale: float, causal: bool):
+    """Gradients (dQ, dK, dV) of L = <Attention(Q,K,V), dO>, fp64.
+
+    GQA: dK/dV of a K/V head are summed over the query heads of its group.
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    dq = np.empty_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            dq[b, h] = _head_backward(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal, dk[b, g], dv[b, g])
+    return dq, dk, dv
+
+
+def head_row_stats(qh, kh, vh, doh, scale: float, causal: bool):
+    """Per-row (lse_i, D_i) of one query head, every row, with D_i = sum_j p_ij dP_ij."""
+    N = qh.shape[0]
+    lse = np.empty(N)
+    Dv = np.empty(N)
+    for c0 in range(0, N, _ROW_CHUNK):
+        r = np.arange(c0, min(N, c0 + _ROW_CHUNK))
+        kcols = (r[-1] + 1) if causal else kh.shape[0]  # columns past the last row are masked anyway
+        s = scores(qh[r], kh[:kcols], scale, r, causal)
+        l = row_lse(s)
+        p = probs(s, l)
+        dp = doh[r] @ vh[:kcols].T
+        lse[r] = l
+        Dv[r] = (p * dp).sum(axis=1)
+    return lse, Dv
+
+
+def attention_backward_sampled(q, k, v, do, scale: float, causal: bool, b: int, hkv: int, q_rows, kv_rows):
+    """Sampled gradients for K/V head (b, hkv) and its query-head group.
+
+    Returns (dq [G, len(q_rows), D], dk [len(kv_rows), D], dv [len(kv_rows), D]),
+    where G = Hq/Hkv query heads of the group in order.  Column j of the
+    gradient needs p_ij and D_i for every row i, so the full per-row
+    statistics of each head are computed first (head_row_stats).
+    """
+    Hq, Hkv = q.shape[1], k.shape[1]
+    G = Hq // Hkv
+    kh, vh = _f64(k[b, hkv]), _f64(v[b, hkv])
+    q_rows = np.asarray(q_rows)
+    kv_rows = np.asarray(kv_rows)
+    N = kh.shape[0]
+    dq = np.empty((G, len(q_rows), kh.shape[1]))
+    dk = np.zeros((len(kv_rows), kh.shape[1]))
+    dv = np.zeros((len(kv_rows), kh.shape[1]))
+    for gi in range(G):
+        h = hkv * G + gi
+        qh, doh = _f64(q[b, h]), _f64(do[b, h])
+        lse, Dv = head_row_stats(qh, kh, vh, doh, scale, causal)
+        # dQ rows: dQ_i = scale * sum_j p_ij (dP_ij - D_i) k_j
+        s = scores(qh[q_rows], kh, scale, q_rows, causal)
+        p = probs(s, lse[q_rows])
+        dp = doh[q_rows] @ vh.T
+        dq[gi] = scale * ((p * (dp - Dv[q_rows][:, None])) @ kh)
+        # dK/dV columns: need every row i (all rows i >= j when causal)
+        allr = np.arange(N)
+        sc = scale * (qh @ kh[kv_rows].T)  # [N, J]
+        if causal:
+            sc = np.where(kv_rows[None, :] > allr[:, None], -np.inf, sc)
+        pc = np.exp(sc - lse[:, None])
+        dpc = doh @ vh[kv_rows].T
+        dsc = pc * (dpc - Dv[:, None])
+        dk += scale * (dsc.T @ qh)
+        dv += pc.T @ doh
+    return dq, dk, dv
+
+
+def attention_forward_blocked(q, k, v, scale: float, causal: bool, block_r: int = 64, block_c: int = 64):
+    """Tiled forward with the online (incremental) softmax, fp64.
+
+    For each row block Q_i and each column block K_j, V_j:
+      S_ij = scale Q_i K_j^T (masked);  m_new = max(m, rowmax S_ij);
+      P~ = exp(S_ij - m_new);  l = exp(m - m_new) l + rowsum P~;
+      O = exp(m - m_new) O + P~ V_j;  m = m_new.
+    Finally O = O / l and lse = m + log l.  Block sizes need not divide N.
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, N))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            kh, vh = k[b, g], v[b, g]
+            for i0 in range(0, N, block_r):
+                rows = np.arange(i0, min(N, i0 + block_r))
+                qi = q[b, h, rows]
+                m = np.full(len(rows), -np.inf)
+                l = np.zeros(len(rows))
+                acc = np.zeros((len(rows), D))
+                for j0 in range(0, N, block_c):
+                    cols = np.arange(j0, min(N, j0 + block_c))
+                    if causal and cols[0] > rows[-1]:
+                        break  # block entirely above the diagonal
+                    s = scale * (qi @ kh[cols].T)
+                    if causal:
+                        s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+                    m_new = np.maximum(m, s.max(axis=1))
+                    pt = np.exp(s - m_new[:, None])
+                    alpha = np.exp(m - m_new)
+                    l = alpha * l + pt.sum(axis=1)
+                    acc = alpha[:, None] * acc + pt @ vh[cols]
+                    m = m_new
+                o[b, h, rows] = acc / l[:, None]
+                lse[b, h, rows] = m + np.log(l)
+    return o, lse
