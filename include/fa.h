@@ -1,0 +1,108 @@
+/*
+ * fa.h — exact tiled (flash) attention for NVIDIA B200 (sm_100a), C ABI.
+ *
+ * What is computed.  For every batch b and query head h (K/V head
+ * g = h / (Hq / Hkv), contiguous groups):
+ *     S = scale * Q K^T            (key j visible to query i iff j <= i when causal)
+ *     P = softmax(S) row-wise,  O = P V,  LSE_i = log sum_j exp(S_ij)  (natural log)
+ * The forward never materialises S or P in global memory: Q is kept on chip
+ * tile by tile while K/V tiles stream past it and an online softmax (running
+ * row max m and running sum l, final O / l correction) accumulates O.  This is
+ * the tiling + incremental softmax of "【词汇专栏】FlashAttention：大模型训练的
+ * 加速器" (sections 2.1, 2.2, 2.3) and of "FlashAttention 在昇腾NPU上到底快在哪"
+ * (sections 二 and 三).
+ * The backward recomputes P from the saved LSE ("FlashAttention V2深度解析：
+ * 反向传播显存优化让大模型训练不再OOM", section 改进1, the recompute-instead-of-
+ * store idea) and uses the closed-form softmax gradient of L = <O, dO>:
+ *     D_i = sum_d dO_id O_id,  dV = P^T dO,  dP = dO V^T,
+ *     dS = P o (dP - D) * scale,  dK = dS^T Q,  dQ = dS K,
+ * with dK/dV of a K/V head summed over the query heads of its group (GQA).
+ * Work is parallel over batch, head and sequence blocks (same deep dive,
+ * section 改进2).
+ *
+ * Layout.  Every tensor is contiguous row-major.
+ *   q, o, dout, dq : bf16 [B, Hq,  N, D]
+ *   k, v, dk, dv   : bf16 [B, Hkv, N, D]
+ *   lse            : fp32 [B, Hq, N]  natural-log log-sum-exp of the scaled logits
+ * Supported: D in {64, 128}; B, Hq, Hkv, N >= 1; Hq % Hkv == 0.  Query and key
+ * lengths are equal (N), so the causal mask is unambiguous.
+ *
+ * Ownership.  The caller allocates and owns every buffer (device memory),
+ * including the backward workspace.  The library allocates no device memory on
+ * these calls.  Pointers must be device pointers aligned to 16 bytes.
+ *
+ * Asynchrony and errors.  Calls enqueue kernels on `stream` and return at
+ * once.  A non-OK status means nothing was launched (argument errors) or the
+ * launch failed (FA_ERR_CUDA).  Outputs are overwritten, never accumulated.
+ * Device-side pipeline waits are bounded; a wait that gives up sets a device
+ * status word that fa_get_device_status() reports (FA_ERR_TIMEOUT).
+ */
+#ifndef TILED_ATTENTION_FA_H
+#define TILED_ATTENTION_FA_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad sizes, bad scale, small workspace */
+    FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, or a non-sm_100 device */
+    FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    FA_ERR_TIMEOUT = 4      /* a device-side pipeline wait gave up (reported by fa_get_device_status) */
+} fa_status;
+
+/* Problem shape.  Hkv == Hq is plain multi-head attention; Hkv < Hq is GQA
+ * (MQA when Hkv == 1).  scale multiplies the logits (1/sqrt(D) is usual); it
+ * must be finite and > 0.  causal != 0 masks key j > query i. */
+typedef struct {
+    int B, Hq, Hkv, N, D;
+    float scale;
+    int causal;
+} fa_shape;
+
+/* Forward.  q [B,Hq,N,D], k/v [B,Hkv,N,D] bf16 in; o [B,Hq,N,D] bf16 and
+ * lse [B,Hq,N] fp32 out.  `stream` is a cudaStream_t (NULL = legacy stream). */
+FA_API fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void* v,
+                 void* o, float* lse, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for `shape` (0 if the shape is invalid):
+ * the per-row statistics (LSE in log2 units and D = rowsum(dO o O), each
+ * padded to a multiple of 128 rows) and an fp32 dQ accumulator [B,Hq,N,D]. */
+FA_API size_t fa_bwd_workspace_bytes(const fa_shape* shape);
+
+/* Backward.  Inputs q, k, v, o, dout (bf16) and lse (fp32, as written by
+ * fa_fwd).  Outputs dq [B,Hq,N,D], dk and dv [B,Hkv,N,D], bf16, overwritten.
+ * `workspace` must be a device buffer of at least fa_bwd_workspace_bytes(shape)
+ * bytes, 256-byte aligned; its contents on entry do not matter. */
+FA_API fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v,
+                 const void* o, const void* dout, const float* lse,
+                 void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reports and clears the device status word of
+ * the current device: FA_ERR_TIMEOUT if any kernel gave up a bounded wait
+ * since the last call, FA_ERR_CUDA if the stream reports an error, else FA_OK. */
+FA_API fa_status fa_get_device_status(void* stream);
+
+/* Static description of a status code. */
+FA_API const char* fa_status_str(fa_status status);
+
+/* Diagnostics: the bitmask of device-side wait sites (bit k = site k) that
+ * the most recent fa_get_device_status() call found and cleared; 0 when
+ * healthy.  Host-only, no CUDA call. */
+FA_API unsigned int fa_debug_timeout_sites(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TILED_ATTENTION_FA_H */

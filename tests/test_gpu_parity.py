@@ -1,0 +1,181 @@
+"""GPU parity: the sm_100a kernels (through the C ABI) against the fp64 oracle.
+
+Tolerances (bf16 inputs and outputs, fp32 accumulation):
+  O     max |O_gpu - O_ref|                 <= 2e-2
+  LSE   max |LSE_gpu - LSE_ref|             <= 1e-3
+  dQ/dK/dV  ||G_gpu - G_ref||_F / ||G_ref||_F <= 2e-2
+Small shapes are compared element by element in full; the five named
+workloads run at full size in the same launch configuration bench.py times,
+and the oracle checks seeded heads (every row of them) or, for the N=65536
+stress case, sampled query and key rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from tiled_attention_16_b200 import attention as A
+from tiled_attention_16_b200.workloads import WORKLOADS, Workload, make_inputs, sample_indices
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, G_TOL = 2e-2, 1e-3, 2e-2
+
+
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    return torch.device("cuda:0")
+
+
+def run(q, k, v, do, causal, scale, backward=True):
+    dev = _gpu()
+    qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
+    o, lse = A.fwd(qd, kd, vd, causal=causal, scale=scale)
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = A.bwd(qd, kd, vd, o, dod, lse, causal=causal, scale=scale)
+        out.update(dq=dq, dk=dk, dv=dv)
+    assert A.device_status() == A.FA_OK, f"device status sites={A.timeout_sites():#x}"
+    return {n: t.float().cpu().double().numpy() for n, t in out.items()}
+
+
+def rel_fro(a, b):
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def assert_fwd(g, o_ref, lse_ref, sel=(slice(None),)):
+    eo = np.abs(g["o"][sel] - o_ref).max()
+    el = np.abs(g["lse"][sel] - lse_ref).max()
+    assert eo <= O_TOL, f"O max abs err {eo}"
+    assert el <= LSE_TOL, f"LSE max abs err {el}"
+
+
+SMALL = [
+    # B, Hq, Hkv, N, D, causal, scale, sigma_qk
+    (1, 2, 2, 128, 64, False, None, 1.0),
+    (1, 2, 2, 128, 64, True, None, 1.0),
+    (2, 3, 3, 17, 64, False, None, 1.0),
+    (2, 3, 3, 17, 128, True, None, 1.0),
+    (1, 2, 2, 1, 128, True, None, 1.0),
+    (1, 2, 2, 1, 64, False, None, 1.0),
+    (1, 4, 2, 300, 128, True, None, 1.0),
+    (1, 4, 2, 257, 128, False, None, 1.0),
+    (1, 8, 1, 384, 64, True, None, 1.0),
+    (2, 2, 2, 513, 128, True, 1.0, 0.3),
+    (1, 2, 2, 640, 128, True, None, 3.0),
+    (1, 2, 2, 1000, 64, False, None, 3.0),
+    (1, 16, 2, 256, 128, False, 0.05, 1.0),
+]
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,N,D,causal,scale,sqk", SMALL)
+def test_small_shapes_full(B, Hq, Hkv, N, D, causal, scale, sqk):
+    wl = Workload("small", B=B, Hq=Hq, Hkv=Hkv, N=N, D=D, causal=causal, seed=1000 + N + D, sigma_qk=sqk, scale=scale)
+    q, k, v, do = make_inputs(wl)
+    sc = wl.softmax_scale
+    g = run(q, k, v, do, causal, sc)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, sc, causal)
+    assert_fwd(g, o_ref, lse_ref)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, sc, causal)
+    for name, ref in (("dq", dq), ("dk", dk), ("dv", dv)):
+        e = rel_fro(g[name], ref)
+        assert e <= G_TOL, f"{name} rel Frobenius err {e}"
+
+
+def test_repeat_calls_identical_forward():
+    wl = WORKLOADS["tiny"].with_(causal=True, N=333)
+    q, k, v, do = make_inputs(wl)
+    a = run(q, k, v, do, True, wl.softmax_scale, backward=False)
+    b = run(q, k, v, do, True, wl.softmax_scale, backward=False)
+    assert np.array_equal(a["o"], b["o"]) and np.array_equal(a["lse"], b["lse"])
+
+
+def _full_size(name, heads, grad_rows=None):
+    """Run workload `name` at full size on the GPU; check the listed (b, h_kv)
+    groups against the oracle: every query head of the group, every row."""
+    wl = WORKLOADS[name]
+    q, k, v, do = make_inputs(wl)
+    sc = wl.softmax_scale
+    g = run(q, k, v, do, wl.causal, sc)
+    G = wl.Hq // wl.Hkv
+    for (b, hk) in heads:
+        hs = slice(hk * G, (hk + 1) * G)
+        qs, ks, vs, dos = q[b:b + 1, hs], k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1], do[b:b + 1, hs]
+        o_ref, lse_ref = oracle.attention_forward(qs, ks, vs, sc, wl.causal)
+        assert_fwd(g, o_ref[0], lse_ref[0], (b, hs))
+        dq, dk, dv = oracle.attention_backward(qs, ks, vs, dos, sc, wl.causal)
+        for nm, gpu, ref in (("dq", g["dq"][b, hs], dq[0]), ("dk", g["dk"][b, hk], dk[0, 0]),
+                             ("dv", g["dv"][b, hk], dv[0, 0])):
+            e = rel_fro(gpu, ref)
+            assert e <= G_TOL, f"{name} (b={b}, hkv={hk}) {nm} rel Frobenius err {e}"
+    for t in ("o", "dq", "dk", "dv"):
+        assert np.isfinite(g[t]).all(), t
+
+
+def test_workload_tiny():
+    wl = WORKLOADS["tiny"]
+    q, k, v, do = make_inputs(wl)
+    g = run(q, k, v, do, wl.causal, wl.softmax_scale)
+    o_ref, lse_ref = oracle.attention_forward(q, k, v, wl.softmax_scale, wl.causal)
+    assert_fwd(g, o_ref, lse_ref)
+    for nm, ref in zip(("dq", "dk", "dv"), oracle.attention_backward(q, k, v, do, wl.softmax_scale, wl.causal)):
+        assert rel_fro(g[nm], ref) <= G_TOL, nm
+
+
+@pytest.mark.timeout(900)
+def test_workload_llama7b():
+    _full_size("llama7b", [(0, 0), (3, 17), (7, 31)])
+
+
+@pytest.mark.timeout(900)
+def test_workload_long():
+    _full_size("long", [(0, 0), (0, 13), (1, 22), (1, 31)])
+
+
+@pytest.mark.timeout(900)
+def test_workload_gqa70b():
+    _full_size("gqa70b", [(0, 0), (0, 7)])
+
+
+@pytest.mark.timeout(1800)
+def test_workload_stress_sampled():
+    wl = WORKLOADS["stress"]
+    q, k, v, do = make_inputs(wl)
+    sc = wl.softmax_scale
+    g = run(q, k, v, do, True, sc)
+    N = wl.N
+    rows = np.array(sample_indices(N, 256, 7, must=(0, 127, 128, 129, N // 2, N - 129, N - 128, N - 1)))
+    for t in ("o", "lse", "dq", "dk", "dv"):
+        assert np.isfinite(g[t]).all(), t
+    for h in (3, 12):
+        o_r, lse_r = oracle.attention_forward_rows(q, k, v, sc, True, 0, h, rows)
+        eo = np.abs(g["o"][0, h, rows] - o_r).max()
+        el = np.abs(g["lse"][0, h, rows] - lse_r).max()
+        assert eo <= O_TOL and el <= LSE_TOL, (h, eo, el)
+        dq_s, dk_s, dv_s = oracle.attention_backward_sampled(q, k, v, do, sc, True, 0, h, rows, rows)
+        for nm, gpu, ref in (("dq", g["dq"][0, h, rows], dq_s[0]), ("dk", g["dk"][0, h, rows], dk_s),
+                             ("dv", g["dv"][0, h, rows], dv_s)):
+            e = rel_fro(gpu, ref)
+            assert e <= G_TOL, f"stress h={h} {nm} rel Frobenius err {e}"
+
+
+def test_lse_consistent_with_output_scale():
+    """Property at any size: with V = I-like one-hot columns the output rows
+    are probability rows, so they sum to 1 and stay in [0, 1]."""
+    dev = _gpu()
+    B, H, N, D = 1, 2, 777, 64
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn(B, H, N, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, H, N, D, generator=g).to(torch.bfloat16)
+    v = torch.zeros(B, H, N, D, dtype=torch.bfloat16)
+    v[..., 0] = 1.0
+    o, lse = A.fwd(q.to(dev), k.to(dev), v.to(dev), causal=True)
+    torch.cuda.synchronize()
+    assert torch.allclose(o[..., 0].float().cpu(), torch.ones(B, H, N), atol=1e-2)
+    assert (o[..., 1:] == 0).all()
+    # causal row 0 sees one key: lse_0 = scale * q_0 . k_0
+    ref0 = (q[..., 0, :].double() * k[..., 0, :].double()).sum(-1) / math.sqrt(D)
+    assert torch.allclose(lse[..., 0].double().cpu(), ref0, atol=1e-3)

@@ -1,0 +1,169 @@
+"""Python binding of the C ABI in include/fa.h (argument marshalling only).
+
+Every step of the attention runs in the sm_100a kernels of
+``libfa_sm100.so``; this module only checks tensors, allocates outputs with
+PyTorch (device memory is PyTorch's job here) and passes raw pointers and the
+current CUDA stream.  There is no fallback: if the library is missing or the
+device is not a B200 the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libfa_sm100.so")
+HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "fa.h")
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+
+
+class FaShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("N", ctypes.c_int),
+                ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int)]
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (built in-tree by ``tiled_attention_16_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing "
+                               "(run `python -m tiled_attention_16_b200.build`)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, sz = ctypes.c_void_p, ctypes.c_size_t
+        shp = ctypes.POINTER(FaShape)
+        L.fa_fwd.argtypes = [shp, vp, vp, vp, vp, vp, vp]
+        L.fa_fwd.restype = ctypes.c_int
+        L.fa_bwd_workspace_bytes.argtypes = [shp]
+        L.fa_bwd_workspace_bytes.restype = sz
+        L.fa_bwd.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.fa_bwd.restype = ctypes.c_int
+        L.fa_get_device_status.argtypes = [vp]
+        L.fa_get_device_status.restype = ctypes.c_int
+        L.fa_status_str.argtypes = [ctypes.c_int]
+        L.fa_status_str.restype = ctypes.c_char_p
+        L.fa_debug_timeout_sites.argtypes = []
+        L.fa_debug_timeout_sites.restype = ctypes.c_uint
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list[str]:
+    """Entry points declared in include/fa.h (FA_API functions)."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    return re.findall(r"FA_API\s+[\w\s\*]+?\b(fa_\w+)\s*\(", text)
+
+
+def status_str(status: int) -> str:
+    return lib().fa_status_str(int(status)).decode()
+
+
+def make_shape(B, Hq, Hkv, N, D, scale, causal) -> FaShape:
+    return FaShape(int(B), int(Hq), int(Hkv), int(N), int(D), float(scale), 1 if causal else 0)
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(t: torch.Tensor, name: str, shape, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _dims(q, k):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, N, D]")
+    B, Hq, N, D = q.shape
+    Hkv = k.shape[1]
+    return B, Hq, Hkv, N, D
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: float | None = None,
+        out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """Attention forward.  Returns (o [B,Hq,N,D] bf16, lse [B,Hq,N] fp32)."""
+    B, Hq, Hkv, N, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(q, "q", (B, Hq, N, D))
+    _check(k, "k", (B, Hkv, N, D))
+    _check(v, "v", (B, Hkv, N, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
+    _check(out, "out", (B, Hq, N, D))
+    _check(lse, "lse", (B, Hq, N), torch.float32)
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    st = lib().fa_fwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr(), _stream_ptr(q.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd")
+    return out, lse
+
+
+def workspace_bytes(B, Hq, Hkv, N, D, causal=False, scale=None) -> int:
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    return int(lib().fa_bwd_workspace_bytes(ctypes.byref(shp)))
+
+
+def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
+        dq=None, dk=None, dv=None, workspace: torch.Tensor | None = None):
+    """Attention backward.  Returns (dq, dk, dv), bf16, shaped like q, k, v."""
+    B, Hq, Hkv, N, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    for t, name, shape in ((q, "q", (B, Hq, N, D)), (k, "k", (B, Hkv, N, D)), (v, "v", (B, Hkv, N, D)),
+                           (o, "o", (B, Hq, N, D)), (do, "do", (B, Hq, N, D))):
+        _check(t, name, shape)
+    _check(lse, "lse", (B, Hq, N), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", (B, Hq, N, D))
+    _check(dk, "dk", (B, Hkv, N, D))
+    _check(dv, "dv", (B, Hkv, N, D))
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    nbytes = int(lib().fa_bwd_workspace_bytes(ctypes.byref(shp)))
+    if workspace is None:
+        workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
+    if workspace.device.type != "cuda" or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    st = lib().fa_bwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                      workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def device_status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the device status word."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    return int(lib().fa_get_device_status(_stream_ptr(dev)))
+
+
+def timeout_sites() -> int:
+    return int(lib().fa_debug_timeout_sites())

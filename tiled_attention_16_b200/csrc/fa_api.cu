@@ -1,0 +1,189 @@
+// fa_api.cu — the C ABI of include/fa.h: argument validation, TMA tensor-map
+// construction and kernel launches on the caller's stream.  No device memory
+// is allocated here; every buffer belongs to the caller.
+#include "fa.h"
+#include "fa_internal.h"
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include <cudaTypedefs.h>
+
+namespace fa {
+
+__device__ unsigned int g_status = 0;
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over a contiguous bf16 [BH, N, D] tensor: box = 64 columns x 128
+// rows x 1 head, 128-byte swizzle; rows past N read as zero.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
+    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTileM), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_shape(const fa_shape* s) {
+    if (!s) return FA_ERR_INVALID_ARG;
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->N < 1 || s->D < 1) return FA_ERR_INVALID_ARG;
+    if (s->Hq % s->Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(s->scale) || !(s->scale > 0.f)) return FA_ERR_INVALID_ARG;
+    // grid and index ranges
+    const long long BH = static_cast<long long>(s->B) * s->Hq;
+    const long long tiles = (static_cast<long long>(s->N) + 255) / 256;
+    if (BH * tiles > 0x7fffffffLL || BH > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+    if (s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+// sm_100 check, cached per device.
+fa_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+    static int cached[64];
+    static std::once_flag once;
+    std::call_once(once, [] { std::memset(cached, 0, sizeof(cached)); });
+    if (dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    if (cached[dev] == 0) {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+            return FA_ERR_CUDA;
+        cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    return cached[dev] == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+unsigned int g_last_sites = 0;
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_str(fa_status s) {
+    switch (s) {
+        case FA_OK: return "ok";
+        case FA_ERR_INVALID_ARG: return "invalid argument";
+        case FA_ERR_UNSUPPORTED: return "unsupported (head dim or device)";
+        case FA_ERR_CUDA: return "CUDA error";
+        case FA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
+                 void* stream) {
+    fa_status st = check_shape(shape);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+    if ((st = check_device()) != FA_OK) return st;
+    const fa_shape& s = *shape;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
+        !make_map(&tv, v, s.B * s.Hkv, s.N, s.D))
+        return FA_ERR_CUDA;
+    FwdParams p;
+    p.B = s.B;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.N = s.N;
+    p.causal = s.causal ? 1 : 0;
+    p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
+    p.n_mblocks = (s.N + 2 * kTileM - 1) / (2 * kTileM);
+    p.o = o;
+    p.lse = lse;
+    cudaError_t e = launch_fwd(s.D, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(const fa_shape* shape) {
+    if (check_shape(shape) != FA_OK) return 0;
+    return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D).total;
+}
+
+fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    fa_status st = check_shape(shape);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_INVALID_ARG;
+    const fa_shape& s = *shape;
+    const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D);
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws.total)
+        return FA_ERR_INVALID_ARG;
+    if ((st = check_device()) != FA_OK) return st;
+    CUtensorMap tq, tk, tv, tdo;
+    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
+        !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D))
+        return FA_ERR_CUDA;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const int Npad = (s.N + kTileM - 1) / kTileM * kTileM;
+    BwdParams p;
+    p.B = s.B;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.N = s.N;
+    p.Npad = Npad;
+    p.causal = s.causal ? 1 : 0;
+    p.scale = s.scale;
+    p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
+    p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2_off);
+    p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec_off);
+    p.dq_acc = reinterpret_cast<float*>(wsb + ws.dq_off);
+    p.dk = dk;
+    p.dv = dv;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
+                                          reinterpret_cast<float*>(wsb + ws.dvec_off), p.dq_acc, s.B * s.Hq, s.N,
+                                          Npad, strm);
+    if (e == cudaSuccess) e = launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm);
+    if (e == cudaSuccess)
+        e = launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_get_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status, sizeof(word)) != cudaSuccess) return FA_ERR_CUDA;
+    g_last_sites = word;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_CUDA;
+        return FA_ERR_TIMEOUT;
+    }
+    return FA_OK;
+}
+
+unsigned int fa_debug_timeout_sites(void) { return g_last_sites; }
+
+}  // extern "C"

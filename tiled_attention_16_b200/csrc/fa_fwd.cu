@@ -1,0 +1,371 @@
+// fa_fwd.cu — tiled attention forward for sm_100a.
+//
+// One CTA owns a work unit of two 128-row query tiles (Q0, Q1) of one
+// (batch, head) and streams the K/V tiles of that head past them, as in the
+// tiling and incremental softmax of "【词汇专栏】FlashAttention：大模型训练的
+// 加速器" (sections 2.1-2.3) and "FlashAttention 在昇腾NPU上到底快在哪"
+// (sections 二, 三): scores are formed one (query tile, key tile) block at a
+// time, multiplied with the V tile at once, and only the running row max m,
+// running sum l and the O accumulator stay on chip.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + correction + epilogue for Q0 (thread = query row)
+//   warps 4-7  the same for Q1
+//   warp  8    MMA issuer (one thread): S = Q K^T and O += P V on tcgen05
+//   warp  9    TMA producer: Q once, K/V through a two-stage ring
+// Tensor memory (512 columns): S0 | S1 | O0 | O1, 128 columns each.  P is
+// written back over the first half of its S block as packed bf16 and read
+// from there as the A operand of the P V MMA.
+//
+// Softmax works in log2 units: p = 2^(s*c - m) with c = scale*log2(e).  The
+// O rescale by 2^(m_old - m_new) is skipped while the row max has grown by at
+// most 8 (p stays <= 256, well inside fp32 / bf16 range); the final O / l and
+// the LSE use the same stale m, so the result is unchanged.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
+
+namespace fa {
+
+namespace {
+
+constexpr int kFwdThreads = 320;
+constexpr int kStages = 2;
+constexpr float kRescaleThreshold = 8.0f;
+
+enum FwdSite { kSiteQ = 0, kSiteK = 1, kSiteV = 2, kSiteKVEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteDrain = 7 };
+
+template <int D>
+struct FwdLayout {
+    static constexpr int kTileBytes = kTileM * D * 2;  // one 128 x D bf16 tile
+    static constexpr int kAtomBytes = kTileM * 128;    // 128 rows x 64 bf16
+    static constexpr int kQ = 0;                        // 2 tiles
+    static constexpr int kK = kQ + 2 * kTileBytes;      // kStages tiles
+    static constexpr int kV = kK + kStages * kTileBytes;
+    static constexpr int kBar = kV + kStages * kTileBytes;
+    static constexpr int kNumBars = 1 + 3 * kStages + 3 * 2 + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
+};
+
+__device__ __forceinline__ float lg2(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Time-bounded wait that ignores the abort flag (used only to drain copies
+// and MMAs that are already in flight before the CTA releases its resources).
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
+    if (mbar_try_wait(bar, parity)) return;
+    unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, 1u << site);
+            return;
+        }
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+              const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using L = FwdLayout<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* q_full = bars + 0;
+    uint64_t* k_full = bars + 1;                 // [kStages]
+    uint64_t* v_full = bars + 1 + kStages;       // [kStages]
+    uint64_t* kv_empty = bars + 1 + 2 * kStages; // [kStages]
+    uint64_t* s_full = bars + 1 + 3 * kStages;   // [2]
+    uint64_t* p_full = s_full + 2;               // [2]
+    uint64_t* o_full = p_full + 2;               // [2]
+    uint64_t* drain = o_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: heaviest (last) query blocks first for causal balance
+    const int BH = p.B * p.Hq;
+    const int mb = p.n_mblocks - 1 - static_cast<int>(blockIdx.x) / BH;
+    const int bh = static_cast<int>(blockIdx.x) % BH;
+    const int b = bh / p.Hq;
+    const int h = bh - b * p.Hq;
+    const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+    const int m0 = mb * 2 * kTileM;
+    const int n_kv_total = (p.N + kTileN - 1) / kTileN;
+    const bool act1 = (m0 + kTileM) < p.N;
+    int nkv[2];
+    if (p.causal) {
+        nkv[0] = 2 * mb + 1;
+        nkv[1] = act1 ? 2 * mb + 2 : 0;
+    } else {
+        nkv[0] = n_kv_total;
+        nkv[1] = act1 ? n_kv_total : 0;
+    }
+    const int n_iter = act1 ? nkv[1] : nkv[0];
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], kTileM);
+            mbar_init(&o_full[s], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const int nsub = act1 ? 2 : 1;
+            mbar_arrive_expect_tx(q_full, nsub * L::kTileBytes);
+            for (int s = 0; s < nsub; ++s)
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kQ + s * L::kTileBytes + a * L::kAtomBytes, &tmQ, q_full, a * 64,
+                                m0 + s * kTileM, bh);
+            int issued = 0;
+            for (int j = 0; j < n_iter; ++j) {
+                const int st = j & 1;
+                if (j >= kStages && !mbar_wait(&kv_empty[st], ((j >> 1) - 1) & 1, abort_flag, kSiteKVEmpty)) break;
+                mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kK + st * L::kTileBytes + a * L::kAtomBytes, &tmK, &k_full[st], a * 64,
+                                j * kTileN, kvh);
+                mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &v_full[st], a * 64,
+                                j * kTileN, kvh);
+                issued = j + 1;
+            }
+            // Make sure no copy is still landing in shared memory when the CTA
+            // leaves (only matters if the pipeline aborted).
+            mbar_wait_drain(q_full, 0, kSiteDrain);
+            for (int j = (issued > kStages ? issued - kStages : 0); j < issued; ++j) {
+                mbar_wait_drain(&k_full[j & 1], (j >> 1) & 1, kSiteDrain);
+                mbar_wait_drain(&v_full[j & 1], (j >> 1) & 1, kSiteDrain);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kTileN, 0, 0);
+            constexpr uint32_t kIdPV = idesc_bf16_f32(kTileM, D, 0, 1);
+            const uint32_t q_base = smem_u32(smem + L::kQ);
+            const uint32_t k_base = smem_u32(smem + L::kK);
+            const uint32_t v_base = smem_u32(smem + L::kV);
+            auto issue_s = [&](int s, int st) {
+                const uint32_t qa = q_base + s * L::kTileBytes;
+                const uint32_t ka = k_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * L::kAtomBytes + (kk & 3) * 32;
+                    mma_ss(tmem + s * 128, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdS,
+                           kk > 0);
+                }
+            };
+            auto issue_pv = [&](int s, int st, int j) {
+                const uint32_t va = v_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk) {
+                    mma_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8,
+                           sdesc_sw128(va + kk * 2048, L::kAtomBytes, 1024), kIdPV, (j > 0 || kk > 0));
+                }
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, kSiteQ) && mbar_wait(&k_full[0], 0, abort_flag, kSiteK);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                tc_commit(&s_full[0]);
+                if (nkv[1] > 0) {
+                    issue_s(1, 0);
+                    tc_commit(&s_full[1]);
+                }
+            }
+            for (int j = 0; ok && j < n_iter; ++j) {
+                const int st = j & 1;
+                const uint32_t ph = (j >> 1) & 1;
+                if (!(ok = mbar_wait(&v_full[st], ph, abort_flag, kSiteV))) break;
+                if (j < nkv[0]) {
+                    if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, kSiteP))) break;
+                    tc_fence_after();
+                    issue_pv(0, st, j);
+                    if (j == nkv[0] - 1) tc_commit(&o_full[0]);
+                    if (j + 1 < nkv[0]) {
+                        if (!(ok = mbar_wait(&k_full[st ^ 1], ((j + 1) >> 1) & 1, abort_flag, kSiteK))) break;
+                        tc_fence_after();
+                        issue_s(0, st ^ 1);
+                        tc_commit(&s_full[0]);
+                    }
+                }
+                if (j < nkv[1]) {
+                    if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, kSiteP))) break;
+                    tc_fence_after();
+                    issue_pv(1, st, j);
+                    if (j == nkv[1] - 1) tc_commit(&o_full[1]);
+                }
+                tc_commit(&kv_empty[st]);
+                if (j + 1 < nkv[1]) {
+                    if (!(ok = mbar_wait(&k_full[st ^ 1], ((j + 1) >> 1) & 1, abort_flag, kSiteK))) break;
+                    tc_fence_after();
+                    issue_s(1, st ^ 1);
+                    tc_commit(&s_full[1]);
+                }
+            }
+            // Wait for every MMA this thread issued before TMEM is released.
+            tc_commit(drain);
+            mbar_wait_drain(drain, 0, kSiteDrain);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int s = warp >> 2;                       // query tile 0 or 1
+        const int r = ((warp & 3) << 5) + lane;        // row inside the tile = TMEM lane
+        const int qrow = m0 + s * kTileM + r;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
+        const uint32_t tS = tmem + lane_off + s * 128;
+        const uint32_t tO = tmem + lane_off + 256 + s * 128;
+        const float c = p.scale_log2;
+        float m_used = -INFINITY;
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv[s]; ++j) {
+            ok = mbar_wait(&s_full[s], j & 1, abort_flag, kSiteS);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+            tmem_ld_wait();
+            float* sv = reinterpret_cast<float*>(&sr[0][0]);
+            const int kv0 = j * kTileN;
+            const bool mask = (p.causal && j == nkv[s] - 1) || (kv0 + kTileN > p.N);
+            if (mask) {
+#pragma unroll
+                for (int cix = 0; cix < 128; ++cix) {
+                    const int kv = kv0 + cix;
+                    if (kv >= p.N || (p.causal && kv > qrow)) sv[cix] = -INFINITY;
+                }
+            }
+            float mx = sv[0];
+#pragma unroll
+            for (int cix = 1; cix < 128; ++cix) mx = fmaxf(mx, sv[cix]);
+            const float m_new = fmaxf(m_used, mx * c);
+            const bool need = (m_new > m_used + kRescaleThreshold);
+            if (__any_sync(0xffffffffu, need)) {
+                const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
+                if (j > 0) {
+#pragma unroll 1
+                    for (int q = 0; q < D / 32; ++q) {
+                        uint32_t orow[32];
+                        tmem_ld32(tO + q * 32, orow);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int t = 0; t < 32; ++t)
+                            orow[t] = __float_as_uint(__uint_as_float(orow[t]) * alpha);
+                        tmem_st32(tO + q * 32, orow);
+                    }
+                }
+                l *= alpha;
+                m_used = m_new;
+            }
+            const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+            uint32_t pk[64];
+            float lsum = 0.f;
+#pragma unroll
+            for (int t = 0; t < 64; ++t) {
+                const float p0 = ex2(fmaf(sv[2 * t], c, -msub));
+                const float p1 = ex2(fmaf(sv[2 * t + 1], c, -msub));
+                lsum += p0 + p1;
+                pk[t] = pack_bf16x2(p0, p1);
+            }
+            l += lsum;
+            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_full[s]);
+        }
+        if (ok && nkv[s] > 0) {
+            ok = mbar_wait(&o_full[s], 0, abort_flag, kSiteO);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const float inv_l = 1.f / l;
+                const bool valid = qrow < p.N;
+                __nv_bfloat16* orow_g =
+                    reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * D;
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + q * 32, ov);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        pk[t] = pack_bf16x2(__uint_as_float(ov[2 * t]) * inv_l, __uint_as_float(ov[2 * t + 1]) * inv_l);
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                    }
+                }
+                if (valid) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + lg2(l)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, cudaStream_t stream) {
+    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.Hq;
+    if (grid == 0) return cudaSuccess;
+    if (D == 128) {
+        auto kern = fa_fwd_kernel<128>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<128>::kAlloc);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kFwdThreads, FwdLayout<128>::kAlloc, stream>>>(tq, tk, tv, p);
+    } else {
+        auto kern = fa_fwd_kernel<64>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, FwdLayout<64>::kAlloc);
+        if (e != cudaSuccess) return e;
+        kern<<<grid, kFwdThreads, FwdLayout<64>::kAlloc, stream>>>(tq, tk, tv, p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace fa

@@ -1,0 +1,53 @@
+// fa_internal.h — launch interface shared by the host API and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+constexpr int kTileM = 128;  // query rows per MMA tile (TMEM lanes)
+constexpr int kTileN = 128;  // key/value rows per tile
+
+struct FwdParams {
+    int B, Hq, Hkv, N;
+    int causal;
+    float scale_log2;  // softmax scale * log2(e)
+    int n_mblocks;     // ceil(N / 256): work unit = two 128-row query tiles
+    void* o;           // bf16 [B,Hq,N,D]
+    float* lse;        // fp32 [B,Hq,N]
+};
+
+struct BwdParams {
+    int B, Hq, Hkv, N, Npad;
+    int causal;
+    float scale;       // softmax scale (dS is pre-multiplied by it)
+    float scale_log2;  // scale * log2(e)
+    const float* lse2; // [B*Hq, Npad] lse * log2(e), +inf on padding rows
+    const float* dvec; // [B*Hq, Npad] D = rowsum(dO o O), 0 on padding rows
+    float* dq_acc;     // [B*Hq, N, D] fp32 accumulator
+    void* dk;          // bf16 [B,Hkv,N,D]
+    void* dv;          // bf16 [B,Hkv,N,D]
+};
+
+// Workspace carve-up for the backward (all offsets 256-byte aligned).
+struct BwdWorkspace {
+    size_t lse2_off, dvec_off, dq_off, total;
+};
+BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D);
+
+cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const FwdParams& p, cudaStream_t stream);
+
+cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse,
+                                  float* lse2, float* dvec, float* dq_acc,
+                                  int BH, int N, int Npad, cudaStream_t stream);
+
+cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
+
+cudaError_t launch_bwd_dq_convert(const float* dq_acc, void* dq, size_t n_elems, cudaStream_t stream);
+
+}  // namespace fa
