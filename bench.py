@@ -1,0 +1,378 @@
+"""Benchmark: tiled attention forward + backward on B200 (one JSON line).
+
+A step is one pass of the whole hot path over one batch: fa_fwd then fa_bwd
+(preprocess, main kernel, dQ convert) on the long-sequence workload
+B=2, Hq=Hkv=32, N=8192, D=128, causal, bf16 (inputs of 128 MiB each, larger
+than the 126 MB L2, so no L2 flush is needed between steps).  FLOPs follow
+the matmul convention: fwd 4*B*H*N^2*D, bwd 10*B*H*N^2*D, causal halved.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long]
+  python bench.py --impl reference ...   # the fp64 CPU oracle as the reference arm
+
+Multi-GPU (torchrun, one rank per GPU): each rank solves its own independent
+problem of the same size (weak scaling, no data-path collective); the timed
+region is bracketed by barriers and the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s on 1 B200 and % of dense BF16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- traffic record
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("fa_bwd.cu", "fa_fwd.cu", "sm100.cuh", "fa_internal.h"):
+        with open(os.path.join(ROOT, "tiled_attention_16_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    rec = d.get(kernel, {}).get(workload)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1])
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def oracle_sample(wl, heads: int):
+    """fp64 oracle forward + backward on `heads` (b, h) heads of the workload.
+    Returns (seconds, flops counted with the same convention, threads)."""
+    import oracle
+    from tiled_attention_16_b200.workloads import make_inputs
+    q, k, v, do = make_inputs(wl.with_(B=1, Hq=heads, Hkv=heads))
+    sc = wl.softmax_scale
+    t0 = time.perf_counter()
+    oracle.attention_forward(q, k, v, sc, wl.causal)
+    oracle.attention_backward(q, k, v, do, sc, wl.causal)
+    dt = time.perf_counter() - t0
+    per_head = (wl.flops_fwd() + wl.flops_bwd()) / (wl.B * wl.Hq)
+    return dt, per_head * heads, blas_threads()
+
+
+def reference_step_sample(wl, q, k, v, do, rows):
+    """One reference step: the oracle's forward and backward terms of a
+    strided sample of query rows of one head (rows spread evenly over the
+    sequence, so their causal cost averages like the whole head's)."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.attention_rows_fwd_bwd(q, k, v, do, wl.softmax_scale, wl.causal, 0, 0, rows)
+    return time.perf_counter() - t0
+
+
+def run_reference(args, wl):
+    import numpy as np
+    from tiled_attention_16_b200.workloads import make_inputs
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    R = min(wl.N, 512)
+    stride = wl.N // R
+    rows = np.arange(stride // 2, wl.N, stride)[:R]
+    q, k, v, do = make_inputs(wl.with_(B=1, Hq=1, Hkv=1))
+    for _ in range(args.warmup):
+        reference_step_sample(wl, q, k, v, do, rows)
+    times = [reference_step_sample(wl, q, k, v, do, rows) for _ in range(args.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    per_head = (wl.flops_fwd() + wl.flops_bwd()) / (wl.B * wl.Hq)
+    flops = per_head * len(rows) / wl.N
+    value = flops / (ms * 1e-3) / 1e12
+    sample = (f"{len(rows)} of {wl.N} query rows (stride {stride}) of 1 of {wl.B * wl.Hq} heads per step, "
+              f"fwd+bwd terms in fp64 (numpy/OpenBLAS)")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, ws),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(wl, ws):
+    return {"workload": f"{wl.name}: B={wl.B} Hq={wl.Hq} Hkv={wl.Hkv} N={wl.N} D={wl.D} "
+                        f"{'causal' if wl.causal else 'non-causal'} bf16 fwd+bwd",
+            "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "N": wl.N, "D": wl.D, "causal": wl.causal,
+            "scale": wl.softmax_scale, "seed": wl.seed,
+            "l2": "inputs larger than L2 (128 MiB per tensor); no flush",
+            "parallelism": f"{ws} independent replica(s), one per GPU"}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_gpu(args, wl):
+    import torch
+    import torch.distributed as dist
+    from tiled_attention_16_b200 import attention as A
+    from tiled_attention_16_b200.build import build
+    from tiled_attention_16_b200.workloads import make_inputs
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    if rank == 0:
+        build()
+    if ws > 1:
+        dist.barrier()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    # inputs resident in HBM (rank r draws its own problem: seed + r)
+    q, k, v, do = (x.to(dev) for x in make_inputs(wl.with_(seed=wl.seed + rank)))
+    o = torch.empty_like(q)
+    lse = torch.empty((wl.B, wl.Hq, wl.N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsb = torch.empty(A.workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.N, wl.D), device=dev, dtype=torch.uint8)
+
+    def step():
+        A.fwd(q, k, v, causal=wl.causal, out=o, lse=lse)
+        A.bwd(q, k, v, o, do, lse, causal=wl.causal, dq=dq, dk=dk, dv=dv, workspace=wsb)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if A.device_status(dev) != A.FA_OK:
+        raise RuntimeError(f"device status not OK after warm-up (sites {A.timeout_sites():#x})")
+
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    sampler.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    A.profile_begin()
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    per_kernel = A.profile_end()
+    if ws > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if A.device_status(dev) != A.FA_OK:
+        raise RuntimeError(f"device status not OK after timing (sites {A.timeout_sites():#x})")
+    ms_total = e0.elapsed_time(e1)
+    if ws > 1:
+        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms = ms_total / args.steps
+    flops_step = wl.flops_fwd() + wl.flops_bwd()
+    value = flops_step * ws / (ms * 1e-3) / 1e12
+
+    # kernel-level numbers from the live events
+    kms = {k: (t / n if n else None) for k, (t, n) in per_kernel.items()}
+    fwd_ms = kms["fa_fwd_kernel"]
+    bwd_ms = sum(x for k, x in kms.items() if k != "fa_fwd_kernel" and x)
+    peaks, peak_src = load_peaks()
+    peak_tf = peaks["bf16_tflops"]
+    bwd_main = kms["fa_bwd_kernel"]
+    # the main backward kernel performs all five backward GEMMs
+    achieved = wl.flops_bwd() / (bwd_main * 1e-3) / 1e12
+    dominant = max(kms, key=lambda k: kms[k] or 0)
+    roofline = {"kernel": "fa_bwd_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": recorded_traffic("fa_bwd_kernel", wl.name),
+                "peak_source": f"{peak_src} bf16_tflops (burst)", "dominant_by_time": dominant,
+                "per_launch_ms": bwd_main}
+    fwd_tf = wl.flops_fwd() / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = wl.flops_bwd() / (bwd_ms * 1e-3) / 1e12
+    pre_bytes = wl.B * wl.Hq * wl.N * (2 * wl.D * 2 + 4 + 8) + wl.B * wl.Hq * wl.N * wl.D * 4
+    conv_bytes = wl.B * wl.Hq * wl.N * wl.D * (4 + 2)
+    breakdown = {
+        "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_of_peak": fwd_tf / peak_tf,
+        "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_of_peak": bwd_tf / peak_tf,
+        "bwd_main_ms": bwd_main,
+        "bwd_preprocess_ms": kms["fa_bwd_preprocess"],
+        "bwd_preprocess_gbs": pre_bytes / (kms["fa_bwd_preprocess"] * 1e-3) / 1e9 if kms["fa_bwd_preprocess"] else None,
+        "bwd_dq_convert_ms": kms["fa_bwd_dq_convert"],
+        "bwd_dq_convert_gbs": conv_bytes / (kms["fa_bwd_dq_convert"] * 1e-3) / 1e9 if kms["fa_bwd_dq_convert"] else None,
+        "hbm_peak_gbs": peaks["hbm_gbs"],
+    }
+    launches = sum(n for _, n in per_kernel.values())
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (x.pin_memory() for x in make_inputs(wl.with_(seed=wl.seed + rank)))
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
+        hdk = torch.empty(dk.shape, dtype=dk.dtype, pin_memory=True)
+        hdv = torch.empty(dv.shape, dtype=dv.dtype, pin_memory=True)
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in (ho, hl, hdq, hdk, hdv))
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            k.copy_(hk, non_blocking=True)
+            v.copy_(hv, non_blocking=True)
+            do.copy_(hdo, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            hdq.copy_(dq, non_blocking=True)
+            hdk.copy_(dk, non_blocking=True)
+            hdv.copy_(dv, non_blocking=True)
+
+        e2e_steps = max(3, min(args.steps, 20))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a0.elapsed_time(a1)
+        if ws > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step * ws / (e_ms / e2e_steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        heads = 4
+        dt, fl, threads = oracle_sample(wl, heads)
+        cpu = {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{heads} of {wl.B * wl.Hq} (b,h) heads, full fwd+bwd in fp64 ({dt:.1f} s)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_of(wl, ws),
+            "frac_of_peak": value / ws / peak_tf, "breakdown": breakdown, "roofline": roofline,
+            "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks, "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    from tiled_attention_16_b200.workloads import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

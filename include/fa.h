@@ -101,6 +101,17 @@ FA_API const char* fa_status_str(fa_status status);
  * healthy.  Host-only, no CUDA call. */
 FA_API unsigned int fa_debug_timeout_sites(void);
 
+/* Per-kernel timing for benchmarks.  After fa_profile_begin(), every kernel
+ * the library launches is bracketed by a pair of CUDA events recorded on the
+ * launching stream.  fa_profile_end() waits for those events, writes for each
+ * kernel kind k the summed duration total_ms[k] and the launch count
+ * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
+ * preprocess, 2 backward main, 3 backward dQ convert (FA_PROFILE_KINDS).
+ * Events are host-created objects; no device memory is allocated. */
+#define FA_PROFILE_KINDS 4
+FA_API fa_status fa_profile_begin(void);
+FA_API fa_status fa_profile_end(float* total_ms, int* launches);
+
 #ifdef __cplusplus
 }
 #endif

@@ -113,23 +113,25 @@ def attention_forward_rows(q, k, v, scale: float, causal: bool, b: int, h: int, 
     return _head_forward(_f64(q[b, h]), _f64(k[b, g]), _f64(v[b, g]), scale, causal, rows)
 
 
-def _head_backward(qh, kh, vh, doh, scale, causal, dk_acc, dv_acc):
+def _head_backward(qh, kh, vh, doh, scale, causal, dk_acc, dv_acc, rows=None):
     """Closed-form gradients of L = <O, dO> for one query head.
 
     dV_j += sum_i p_ij dO_i;  dP_ij = dO_i . v_j;  D_i = sum_j p_ij dP_ij;
     dS_ij = p_ij (dP_ij - D_i);  dQ_i = scale sum_j dS_ij k_j;
     dK_j += scale sum_i dS_ij q_i.
+    With `rows` given, only those query rows contribute (their dQ rows are
+    returned, in order, and their terms are added to dK/dV); by default all.
     """
-    N = qh.shape[0]
-    dq = np.empty_like(qh)
-    for c0 in range(0, N, _ROW_CHUNK):
-        r = np.arange(c0, min(N, c0 + _ROW_CHUNK))
+    rows = np.arange(qh.shape[0]) if rows is None else np.asarray(rows)
+    dq = np.empty((len(rows), qh.shape[1]))
+    for c0 in range(0, len(rows), _ROW_CHUNK):
+        r = rows[c0:c0 + _ROW_CHUNK]
         s = scores(qh[r], kh, scale, r, causal)
         p = probs(s, row_lse(s))
         dp = doh[r] @ vh.T
         Di = (p * dp).sum(axis=1)
         ds = p * (dp - Di[:, None])
-        dq[r] = scale * (ds @ kh)
+        dq[c0:c0 + len(r)] = scale * (ds @ kh)
         dk_acc += scale * (ds.T @ qh[r])
         dv_acc += p.T @ doh[r]
     return dq
@@ -151,6 +153,21 @@ def attention_backward(q, k, v, do, scale: float, causal: bool):
             g = kv_head_of(h, Hq, Hkv)
             dq[b, h] = _head_backward(q[b, h], k[b, g], v[b, g], do[b, h], scale, causal, dk[b, g], dv[b, g])
     return dq, dk, dv
+
+
+def attention_rows_fwd_bwd(q, k, v, do, scale: float, causal: bool, b: int, h: int, rows):
+    """Forward and backward terms of the listed query rows of head (b, h):
+    (o_rows, lse_rows, dq_rows, dk_part, dv_part), where dk_part/dv_part are
+    the contributions of those rows to dK/dV of the head's K/V head.  Summing
+    the parts over a partition of the rows gives the full dK/dV."""
+    Hq, Hkv = q.shape[1], k.shape[1]
+    g = kv_head_of(h, Hq, Hkv)
+    qh, kh, vh, doh = _f64(q[b, h]), _f64(k[b, g]), _f64(v[b, g]), _f64(do[b, h])
+    o_r, lse_r = _head_forward(qh, kh, vh, scale, causal, rows)
+    dk = np.zeros_like(kh)
+    dv = np.zeros_like(vh)
+    dq_r = _head_backward(qh, kh, vh, doh, scale, causal, dk, dv, rows)
+    return o_r, lse_r, dq_r, dk, dv
 
 
 def head_row_stats(qh, kh, vh, doh, scale: float, causal: bool):

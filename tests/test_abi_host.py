@@ -18,7 +18,7 @@ build()
 def test_exports_every_declared_symbol():
     names = A.declared_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
-                          "fa_status_str", "fa_debug_timeout_sites"}
+                          "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -116,3 +116,11 @@ def test_python_binding_rejects_cpu_tensors():
     q = torch.zeros(1, 2, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         A.fwd(q, q, q)
+
+
+def test_profile_hooks_without_launches():
+    A.profile_begin()
+    res = A.profile_end()
+    assert set(res) == set(A.PROFILE_KINDS)
+    assert all(v == (0.0, 0) for v in res.values())
+    assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG

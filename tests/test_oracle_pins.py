@@ -346,6 +346,28 @@ def test_sampled_functions_match_full(causal):
             np.testing.assert_allclose(dv_s, dv[b, g, rows], atol=1e-11)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_partition_sums_to_full(causal):
+    q, k, v, do = rand_qkv(1, 2, 1, 90, 6, 170)
+    o, lse = oracle.attention_forward(q, k, v, 0.4, causal)
+    dq, dk, dv = oracle.attention_backward(q, k, v, do, 0.4, causal)
+    parts = [np.arange(0, 90, 3), np.arange(1, 90, 3), np.arange(2, 90, 3)]
+    for h in range(2):
+        dk_sum = np.zeros_like(dk[0, 0])
+        dv_sum = np.zeros_like(dv[0, 0])
+        for rows in parts:
+            o_r, l_r, dq_r, dk_p, dv_p = oracle.attention_rows_fwd_bwd(q, k, v, do, 0.4, causal, 0, h, rows)
+            np.testing.assert_allclose(o_r, o[0, h, rows], atol=1e-12)
+            np.testing.assert_allclose(l_r, lse[0, h, rows], atol=1e-12)
+            np.testing.assert_allclose(dq_r, dq[0, h, rows], atol=1e-12)
+            dk_sum += dk_p
+            dv_sum += dv_p
+        if h == 0:
+            dk0, dv0 = dk_sum, dv_sum
+    np.testing.assert_allclose(dk0 + dk_sum, dk[0, 0], atol=1e-11)
+    np.testing.assert_allclose(dv0 + dv_sum, dv[0, 0], atol=1e-11)
+
+
 # ---------------------------------------------------------------- inputs
 def test_workload_inputs_are_seeded_bf16():
     wl = WORKLOADS["tiny"]

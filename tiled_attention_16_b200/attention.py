@@ -58,6 +58,10 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_debug_timeout_sites.argtypes = []
         L.fa_debug_timeout_sites.restype = ctypes.c_uint
+        L.fa_profile_begin.argtypes = []
+        L.fa_profile_begin.restype = ctypes.c_int
+        L.fa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
+        L.fa_profile_end.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -167,3 +171,22 @@ def device_status(device=None) -> int:
 
 def timeout_sites() -> int:
     return int(lib().fa_debug_timeout_sites())
+
+
+PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert")
+
+
+def profile_begin() -> None:
+    st = lib().fa_profile_begin()
+    if st != FA_OK:
+        raise FAError(st, "fa_profile_begin")
+
+
+def profile_end() -> dict:
+    """{kernel name: (total ms, launches)} for the launches since profile_begin()."""
+    ms = (ctypes.c_float * 4)()
+    n = (ctypes.c_int * 4)()
+    st = lib().fa_profile_end(ms, n)
+    if st != FA_OK:
+        raise FAError(st, "fa_profile_end")
+    return {k: (float(ms[i]), int(n[i])) for i, k in enumerate(PROFILE_KINDS)}

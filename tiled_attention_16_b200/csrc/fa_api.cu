@@ -8,6 +8,8 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
+#include <vector>
 
 #include <cudaTypedefs.h>
 
@@ -80,6 +82,50 @@ fa_status check_device() {
 
 unsigned int g_last_sites = 0;
 
+// ---- optional per-kernel event timing (fa_profile_begin / fa_profile_end)
+struct Profiler {
+    std::mutex mu;
+    bool on = false;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pool;
+    std::vector<int> kind;  // kind of each used pair
+    size_t used = 0;
+};
+Profiler& prof() {
+    static Profiler p;
+    return p;
+}
+
+// Returns the event pair to bracket the next launch of `kind`, or null events
+// when profiling is off.
+std::pair<cudaEvent_t, cudaEvent_t> prof_pair(int kind) {
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> g(p.mu);
+    if (!p.on) return {nullptr, nullptr};
+    if (p.used == p.pool.size()) {
+        if (p.pool.size() >= (1u << 20)) return {nullptr, nullptr};
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return {nullptr, nullptr};
+        if (cudaEventCreate(&b) != cudaSuccess) {
+            cudaEventDestroy(a);
+            return {nullptr, nullptr};
+        }
+        p.pool.emplace_back(a, b);
+        p.kind.push_back(kind);
+    }
+    p.kind[p.used] = kind;
+    return p.pool[p.used++];
+}
+
+// Launch `fn` on `s`, bracketed by profiling events when enabled.
+template <class F>
+cudaError_t timed(int kind, cudaStream_t s, F&& fn) {
+    auto ev = prof_pair(kind);
+    if (ev.first) cudaEventRecord(ev.first, s);
+    cudaError_t e = fn();
+    if (ev.second) cudaEventRecord(ev.second, s);
+    return e;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -119,7 +165,8 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.n_mblocks = (s.N + 2 * kTileM - 1) / (2 * kTileM);
     p.o = o;
     p.lse = lse;
-    cudaError_t e = launch_fwd(s.D, tq, tk, tv, p, static_cast<cudaStream_t>(stream));
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -162,12 +209,16 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.dk = dk;
     p.dv = dv;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    cudaError_t e = launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
-                                          reinterpret_cast<float*>(wsb + ws.dvec_off), p.dq_acc, s.B * s.Hq, s.N,
-                                          Npad, strm);
-    if (e == cudaSuccess) e = launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm);
+    cudaError_t e = timed(1, strm, [&] {
+        return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
+                                     reinterpret_cast<float*>(wsb + ws.dvec_off), p.dq_acc, s.B * s.Hq, s.N, Npad,
+                                     strm);
+    });
+    if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
     if (e == cudaSuccess)
-        e = launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
+        e = timed(3, strm, [&] {
+            return launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
+        });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -185,5 +236,40 @@ fa_status fa_get_device_status(void* stream) {
 }
 
 unsigned int fa_debug_timeout_sites(void) { return g_last_sites; }
+
+fa_status fa_profile_begin(void) {
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.on = true;
+    p.used = 0;
+    return FA_OK;
+}
+
+fa_status fa_profile_end(float* total_ms, int* launches) {
+    Profiler& p = prof();
+    std::lock_guard<std::mutex> g(p.mu);
+    p.on = false;
+    if (!total_ms || !launches) return FA_ERR_INVALID_ARG;
+    for (int k = 0; k < FA_PROFILE_KINDS; ++k) {
+        total_ms[k] = 0.f;
+        launches[k] = 0;
+    }
+    fa_status st = FA_OK;
+    for (size_t i = 0; i < p.used; ++i) {
+        if (cudaEventSynchronize(p.pool[i].second) != cudaSuccess) {
+            st = FA_ERR_CUDA;
+            continue;
+        }
+        float ms = 0.f;
+        if (cudaEventElapsedTime(&ms, p.pool[i].first, p.pool[i].second) != cudaSuccess) {
+            st = FA_ERR_CUDA;
+            continue;
+        }
+        total_ms[p.kind[i]] += ms;
+        launches[p.kind[i]] += 1;
+    }
+    p.used = 0;
+    return st;
+}
 
 }  // extern "C"
