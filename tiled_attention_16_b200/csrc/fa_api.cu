@@ -163,6 +163,13 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.causal = s.causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
     p.n_mblocks = (s.N + 2 * kTileM - 1) / (2 * kTileM);
+    // Query heads per scheduling group: keep the K/V streamed by the group's
+    // resident CTAs within ~32 MiB of L2.
+    {
+        const double per_head = 4.0 * s.N * s.D / (s.Hq / s.Hkv);
+        const int g = static_cast<int>(32.0 * 1024 * 1024 / per_head);
+        p.heads_per_group = g < 1 ? 1 : (g > s.B * s.Hq ? s.B * s.Hq : g);
+    }
     p.o = o;
     p.lse = lse;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
@@ -201,9 +208,16 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.N = s.N;
     p.Npad = Npad;
     p.causal = s.causal ? 1 : 0;
+    // K/V heads per scheduling group: keep the group's Q, dO (bf16) and dQ
+    // accumulator (fp32) of all its query heads within ~48 MiB of L2.
+    {
+        const double per_kv_head = 8.0 * s.N * s.D * (s.Hq / s.Hkv);
+        const int g = static_cast<int>(48.0 * 1024 * 1024 / per_kv_head);
+        p.heads_per_group = g < 1 ? 1 : (g > s.B * s.Hkv ? s.B * s.Hkv : g);
+    }
     p.scale = s.scale;
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
-    p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2_off);
+    p.lse2 =reinterpret_cast<const float*>(wsb + ws.lse2_off);
     p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec_off);
     p.dq_acc = reinterpret_cast<float*>(wsb + ws.dq_off);
     p.dk = dk;

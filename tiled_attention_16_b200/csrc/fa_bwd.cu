@@ -12,22 +12,30 @@
 //   1. fa_bwd_preprocess: D_i = sum_d dO_id O_id and lse2_i = lse_i*log2(e)
 //      (both padded to a multiple of 128 rows: D = 0, lse2 = +inf, so padded
 //      query rows get P = 0), and zeroes the fp32 dQ accumulator.  HBM-bound.
-//   2. fa_bwd_kernel: one CTA per (batch, K/V head, 128-row key block).  K_j
-//      and V_j stay in shared memory; the CTA walks every query head of the
-//      GQA group and every query tile i (i >= j when causal):
+//   2. fa_bwd_kernel: one CTA per (batch, K/V head, 128-row key block j).
+//      K_j and V_j stay in shared memory; Q_i / dO_i tiles stream through a
+//      two-stage ring while the CTA walks every query head of the GQA group
+//      and every query tile i (i >= j when causal):
 //        S^T = K_j Q_i^T,  P^T = 2^(S^T c - lse2),  dP^T = V_j dO_i^T,
 //        dV += P^T dO_i,   dS^T = P^T o (dP^T - D) * scale,
-//        dK += dS^T Q_i,   dQ_i += dS K_j  (fp32 vector atomics).
+//        dK += dS^T Q_i,   dQ_i += dS K_j  (fp32 reductions into global).
 //      dK/dV accumulate in tensor memory over the whole group, so GQA needs
-//      no atomics for them.
+//      no atomics for them.  With D = 128 the dQ tile is computed transposed,
+//      dQ^T = K_j^T dS^T, so a warp's reduction covers one 128-byte line.
 //   3. fa_bwd_dq_convert: dQ = bf16(dQ accumulator).  HBM-bound.
 //
 // Warp roles of fa_bwd_kernel (320 threads):
-//   warps 0-3  P / dS (thread = key row = TMEM lane), then the dK/dV epilogue
-//   warps 4-7  dQ drain (thread = query row = TMEM lane): TMEM -> atomics
+//   warps 0-7  compute: thread = key row (TMEM lane); warps 0-3 take query
+//              columns 0-63, warps 4-7 columns 64-127.  Per query tile they
+//              form P^T, drain the previous dQ tile, then form dS^T; at the
+//              end they write dK and dV.
 //   warp  8    MMA issuer (one thread)
 //   warp  9    TMA producer
-// Tensor memory: S^T (P^T over its first half) | dP^T, later dQ | dV | dK.
+// Tensor memory: S^T (P^T over its first half) | dP^T, then dQ | dV | dK.
+// MMA issue order per query tile it:
+//   S(it) ; dK(it-1), dQ(it-1) ; dP(it) ; dV(it)
+// so the tensor core works on S and dK/dQ while the compute warps form P and
+// dS, and dP(it) waits only for the drain of dQ(it-1) (they share columns).
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -38,10 +46,12 @@ namespace fa {
 namespace {
 
 constexpr int kBwdThreads = 320;
+constexpr int kCompute = 256;  // compute threads (warps 0-7)
+constexpr int kMaxDynSmem = 232448;
 
 enum BwdSite {
     kBSiteKV = 8, kBSiteQ = 9, kBSiteDO = 10, kBSiteQEmpty = 11, kBSiteDOEmpty = 12, kBSiteS = 13,
-    kBSiteDP = 14, kBSiteP = 15, kBSiteDS = 16, kBSiteDSEmpty = 17, kBSiteDQ = 18, kBSiteDQFree = 19,
+    kBSiteDP = 14, kBSiteP = 15, kBSiteDS = 16, kBSiteSmem = 17, kBSiteDQ = 18, kBSiteDQFree = 19,
     kBSiteDKV = 20, kBSiteDrain = 21
 };
 
@@ -51,16 +61,19 @@ struct BwdLayout {
     static constexpr int kAtomBytes = kTileM * 128;
     static constexpr int kK = 0;
     static constexpr int kV = kK + kTileBytes;
-    static constexpr int kQ = kV + kTileBytes;
-    static constexpr int kDO = kQ + kTileBytes;
-    static constexpr int kDS = kDO + kTileBytes;         // 128 x 128 bf16
-    static constexpr int kLse = kDS + kTileM * kTileN * 2;  // 128 fp32
-    static constexpr int kDvec = kLse + kTileN * 4;        // 128 fp32
-    static constexpr int kBar = kDvec + kTileN * 4;
+    static constexpr int kQ = kV + kTileBytes;          // 2 stages
+    static constexpr int kDO = kQ + 2 * kTileBytes;     // 2 stages
+    static constexpr int kDS = kDO + 2 * kTileBytes;    // 128 x 128 bf16
+    static constexpr int kLse = kDS + kTileM * kTileN * 2;  // 2 stages x 128 fp32
+    static constexpr int kDvec = kLse + 2 * kTileN * 4;    // 2 stages x 128 fp32
+    static constexpr int kBar = kDvec + 2 * kTileN * 4;
     static constexpr int kNumBars = 16;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
-    static constexpr int kAlloc = kBytes + 1024;
+    // Request room for base alignment when it fits; the kernel checks the
+    // actual slack at run time.
+    static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
+    static_assert(kBytes <= kMaxDynSmem, "backward shared memory layout too large");
 };
 
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, int site) {
@@ -73,6 +86,14 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
             return;
         }
     }
+}
+
+__device__ __forceinline__ void red_add_f32(float* addr, float v) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d) : "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -149,54 +170,70 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
               const BwdParams p) {
     using L = BwdLayout<D>;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // dQ^T (lanes = head dim) when D fills all 128 lanes, else dQ (lanes = query rows)
+    constexpr bool kDQT = (D == 128);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+    if (pad + L::kBytes > static_cast<uint32_t>(L::kAlloc)) {
+        // Not enough slack to align the swizzled tiles: report and leave
+        // before touching any barrier or tensor memory (uniform for the CTA).
+        if (threadIdx.x == 0) atomicOr(&g_status, 1u << kBSiteSmem);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* q_full = bars + 1;
-    uint64_t* do_full = bars + 2;
-    uint64_t* q_empty = bars + 3;
-    uint64_t* do_empty = bars + 4;
-    uint64_t* s_full = bars + 5;
-    uint64_t* dp_full = bars + 6;
-    uint64_t* p_full = bars + 7;
-    uint64_t* ds_full = bars + 8;
-    uint64_t* ds_empty = bars + 9;
-    uint64_t* dq_full = bars + 10;
-    uint64_t* dq_free = bars + 11;
-    uint64_t* dkv_full = bars + 12;
-    uint64_t* drain = bars + 13;
+    uint64_t* q_full = bars + 1;    // [2]
+    uint64_t* q_empty = bars + 3;   // [2]
+    uint64_t* do_full = bars + 5;   // [2]
+    uint64_t* do_empty = bars + 7;  // [2]
+    uint64_t* s_full = bars + 9;
+    uint64_t* dp_full = bars + 10;
+    uint64_t* p_full = bars + 11;
+    uint64_t* ds_full = bars + 12;
+    uint64_t* dq_full = bars + 13;
+    uint64_t* dq_free = bars + 14;
+    uint64_t* dkv_full = bars + 15;
+    uint64_t* drain = reinterpret_cast<uint64_t*>(smem + L::kMisc + 8);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: key block j of (b, kv head); lightest-last for causal
+    // ---- work unit: head groups; inside a group, key block j ascending
+    //      (heaviest first when causal), then head
     const int BHkv = p.B * p.Hkv;
-    const int j = static_cast<int>(blockIdx.x) / BHkv;
-    const int bkv = static_cast<int>(blockIdx.x) % BHkv;
+    const int T = (p.N + kTileM - 1) / kTileM;
+    const int tile = static_cast<int>(blockIdx.x);
+    const int grp = tile / (p.heads_per_group * T);
+    const int h0 = grp * p.heads_per_group;
+    const int nh = min(p.heads_per_group, BHkv - h0);
+    const int rr = tile - grp * p.heads_per_group * T;
+    const int j = rr / nh;
+    const int bkv = h0 + (rr - j * nh);
     const int b = bkv / p.Hkv;
     const int hkv = bkv - b * p.Hkv;
     const int G = p.Hq / p.Hkv;
-    const int T = (p.N + kTileM - 1) / kTileM;
     const int i0 = p.causal ? j : 0;
     const int per_head = T - i0;
     const int n_it = G * per_head;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
-        mbar_init(q_full, 1);
-        mbar_init(do_full, 1);
-        mbar_init(q_empty, 1);
-        mbar_init(do_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&do_full[s], 1);
+            mbar_init(&do_empty[s], 1);
+        }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(p_full, kTileN);
-        mbar_init(ds_full, kTileN);
-        mbar_init(ds_empty, 1);
+        mbar_init(p_full, kCompute);
+        mbar_init(ds_full, kCompute);
         mbar_init(dq_full, 1);
-        mbar_init(dq_free, kTileM);
+        mbar_init(dq_free, kCompute);
         mbar_init(dkv_full, 1);
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -226,33 +263,39 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             int issued_q = 0, issued_do = 0;
             for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
                 const int g = it / per_head;
                 const int i = i0 + (it - g * per_head);
                 const int bhq = b * p.Hq + hkv * G + g;
-                if (it > 0 && !mbar_wait(q_empty, (it - 1) & 1, abort_flag, kBSiteQEmpty)) break;
-                mbar_arrive_expect_tx(q_full, L::kTileBytes + 2 * kTileM * 4);
+                if (it >= 2 && !mbar_wait(&q_empty[st], ((it >> 1) - 1) & 1, abort_flag, kBSiteQEmpty)) break;
+                mbar_arrive_expect_tx(&q_full[st], L::kTileBytes + 2 * kTileM * 4);
                 for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kQ + a * L::kAtomBytes, &tmQ, q_full, a * 64, i * kTileM, bhq);
+                    tma_load_3d(smem + L::kQ + st * L::kTileBytes + a * L::kAtomBytes, &tmQ, &q_full[st], a * 64,
+                                i * kTileM, bhq);
                 const size_t srow = static_cast<size_t>(bhq) * p.Npad + static_cast<size_t>(i) * kTileM;
-                bulk_load(smem + L::kLse, p.lse2 + srow, kTileM * 4, q_full);
-                bulk_load(smem + L::kDvec, p.dvec + srow, kTileM * 4, q_full);
+                bulk_load(smem + L::kLse + st * kTileM * 4, p.lse2 + srow, kTileM * 4, &q_full[st]);
+                bulk_load(smem + L::kDvec + st * kTileM * 4, p.dvec + srow, kTileM * 4, &q_full[st]);
                 issued_q = it + 1;
-                if (it > 0 && !mbar_wait(do_empty, (it - 1) & 1, abort_flag, kBSiteDOEmpty)) break;
-                mbar_arrive_expect_tx(do_full, L::kTileBytes);
+                if (it >= 2 && !mbar_wait(&do_empty[st], ((it >> 1) - 1) & 1, abort_flag, kBSiteDOEmpty)) break;
+                mbar_arrive_expect_tx(&do_full[st], L::kTileBytes);
                 for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kDO + a * L::kAtomBytes, &tmDO, do_full, a * 64, i * kTileM, bhq);
+                    tma_load_3d(smem + L::kDO + st * L::kTileBytes + a * L::kAtomBytes, &tmDO, &do_full[st], a * 64,
+                                i * kTileM, bhq);
                 issued_do = it + 1;
             }
             mbar_wait_drain(kv_full, 0, kBSiteDrain);
-            if (issued_q > 0) mbar_wait_drain(q_full, (issued_q - 1) & 1, kBSiteDrain);
-            if (issued_do > 0) mbar_wait_drain(do_full, (issued_do - 1) & 1, kBSiteDrain);
+            for (int it = (issued_q > 2 ? issued_q - 2 : 0); it < issued_q; ++it)
+                mbar_wait_drain(&q_full[it & 1], (it >> 1) & 1, kBSiteDrain);
+            for (int it = (issued_do > 2 ? issued_do - 2 : 0); it < issued_do; ++it)
+                mbar_wait_drain(&do_full[it & 1], (it >> 1) & 1, kBSiteDrain);
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdSq = idesc_bf16_f32(kTileN, kTileM, 0, 0);  // S^T, dP^T: K-major both
             constexpr uint32_t kIdAcc = idesc_bf16_f32(kTileN, D, 0, 1);      // dV, dK: A K-major, B MN-major
-            constexpr uint32_t kIdDQ = idesc_bf16_f32(kTileM, D, 1, 1);       // dQ: both MN-major
+            // dQ^T = K^T dS^T (M = D, N = query) or dQ = dS K (M = query, N = D); both operands MN-major
+            constexpr uint32_t kIdDQ = kDQT ? idesc_bf16_f32(D, kTileM, 1, 1) : idesc_bf16_f32(kTileM, D, 1, 1);
             const uint32_t k_base = smem_u32(smem + L::kK);
             const uint32_t v_base = smem_u32(smem + L::kV);
             const uint32_t q_base = smem_u32(smem + L::kQ);
@@ -260,28 +303,58 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             const uint32_t ds_base = smem_u32(smem + L::kDS);
             constexpr uint32_t kAtom = L::kAtomBytes;
             constexpr uint32_t kDsAtom = kTileN * 128;  // dS^T: 64 query columns x 128 key rows
+            auto issue_dk_dq = [&](int it_prev) {
+                const uint32_t qa = q_base + (it_prev & 1) * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTileM / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kDsAtom + (kk & 3) * 32;
+                    mma_ss(tmem + kColDK, sdesc_sw128(ds_base + off, 16, 1024),
+                           sdesc_sw128(qa + kk * 2048, kAtom, 1024), kIdAcc, (it_prev > 0 || kk > 0));
+                }
+                tc_commit(&q_empty[it_prev & 1]);
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk) {
+                    const uint64_t kdesc = sdesc_sw128(k_base + kk * 2048, kAtom, 1024);
+                    const uint64_t dsdesc = sdesc_sw128(ds_base + kk * 2048, kDsAtom, 1024);
+                    if constexpr (kDQT)
+                        mma_ss(tmem + kColDP, kdesc, dsdesc, kIdDQ, kk > 0);
+                    else
+                        mma_ss(tmem + kColDP, dsdesc, kdesc, kIdDQ, kk > 0);
+                }
+                tc_commit(dq_full);
+            };
             bool ok = mbar_wait(kv_full, 0, abort_flag, kBSiteKV);
             for (int it = 0; ok && it < n_it; ++it) {
+                const int st = it & 1;
+                const uint32_t sph = (it >> 1) & 1;
                 const uint32_t ph = it & 1;
                 // S^T = K Q^T
-                if (!(ok = mbar_wait(q_full, ph, abort_flag, kBSiteQ))) break;
+                if (!(ok = mbar_wait(&q_full[st], sph, abort_flag, kBSiteQ))) break;
                 tc_fence_after();
+                const uint32_t qa = q_base + st * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    mma_ss(tmem + kColS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(q_base + off, 16, 1024),
-                           kIdSq, kk > 0);
+                    mma_ss(tmem + kColS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), kIdSq,
+                           kk > 0);
                 }
                 tc_commit(s_full);
-                // dP^T = V dO^T  (into the dQ columns: the previous dQ must be drained)
-                if (!(ok = mbar_wait(do_full, ph, abort_flag, kBSiteDO))) break;
+                // dK, dQ of the previous query tile
+                if (it > 0) {
+                    if (!(ok = mbar_wait(ds_full, ph ^ 1, abort_flag, kBSiteDS))) break;
+                    tc_fence_after();
+                    issue_dk_dq(it - 1);
+                }
+                // dP^T = V dO^T (its columns hold dQ until the compute warps drained it)
+                if (!(ok = mbar_wait(&do_full[st], sph, abort_flag, kBSiteDO))) break;
                 if (it > 0 && !(ok = mbar_wait(dq_free, ph ^ 1, abort_flag, kBSiteDQFree))) break;
                 tc_fence_after();
+                const uint32_t da = do_base + st * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    mma_ss(tmem + kColDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(do_base + off, 16, 1024),
-                           kIdSq, kk > 0);
+                    mma_ss(tmem + kColDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), kIdSq,
+                           kk > 0);
                 }
                 tc_commit(dp_full);
                 // dV += P^T dO   (P^T from TMEM, dO as an MN-major B operand)
@@ -289,89 +362,131 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTileM / 16; ++kk)
-                    mma_ts(tmem + kColDV, tmem + kColS + kk * 8, sdesc_sw128(do_base + kk * 2048, kAtom, 1024), kIdAcc,
+                    mma_ts(tmem + kColDV, tmem + kColS + kk * 8, sdesc_sw128(da + kk * 2048, kAtom, 1024), kIdAcc,
                            (it > 0 || kk > 0));
-                tc_commit(do_empty);
-                // dK += dS^T Q ; dQ = dS K
-                if (!(ok = mbar_wait(ds_full, ph, abort_flag, kBSiteDS))) break;
-                tc_fence_after();
-#pragma unroll
-                for (int kk = 0; kk < kTileM / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kDsAtom + (kk & 3) * 32;
-                    mma_ss(tmem + kColDK, sdesc_sw128(ds_base + off, 16, 1024),
-                           sdesc_sw128(q_base + kk * 2048, kAtom, 1024), kIdAcc, (it > 0 || kk > 0));
-                }
-                tc_commit(q_empty);
-#pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk)
-                    mma_ss(tmem + kColDP, sdesc_sw128(ds_base + kk * 2048, kDsAtom, 1024),
-                           sdesc_sw128(k_base + kk * 2048, kAtom, 1024), kIdDQ, kk > 0);
-                tc_commit(dq_full);
-                tc_commit(ds_empty);
+                tc_commit(&do_empty[st]);
             }
-            if (ok) tc_commit(dkv_full);
+            if (ok && n_it > 0) {
+                if (mbar_wait(ds_full, (n_it - 1) & 1, abort_flag, kBSiteDS)) {
+                    tc_fence_after();
+                    issue_dk_dq(n_it - 1);
+                    tc_commit(dkv_full);
+                }
+            }
             tc_commit(drain);
             mbar_wait_drain(drain, 0, kBSiteDrain);
         }
-    } else if (warp < 4) {
-        // ------------------------------------------------------------ P / dS
-        const int r = (warp << 5) + lane;  // key row inside the block = TMEM lane
+    } else {
+        // ------------------------------------------------------------ compute (P, dQ drain, dS)
+        const int wg = warp >> 2;                   // query-column half
+        const int wq = warp & 3;                    // TMEM lane quarter
+        const int r = (wq << 5) + lane;             // key row of the block = TMEM lane
         const int kv = j * kTileN + r;
-        const uint32_t lane_off = static_cast<uint32_t>(warp << 5) << 16;
+        const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
+        const int c0 = wg * 64;                     // first query column of this half
         const float c = p.scale_log2;
-        const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse);
-        const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec);
         uint8_t* ds_s = smem + L::kDS;
+        const bool kv_ok = kv < p.N;
+        float pv[64];
+
+        // dQ tile of query tile `itp` (TMEM) -> fp32 reductions into the accumulator.
+        auto drain_dq = [&](int itp) -> bool {
+            if (!mbar_wait(dq_full, itp & 1, abort_flag, kBSiteDQ)) return false;
+            tc_fence_after();
+            const int g = itp / per_head;
+            const int i = i0 + (itp - g * per_head);
+            const int bhq = b * p.Hq + hkv * G + g;
+            if constexpr (kDQT) {
+                // lanes = head-dim index d = r, columns = query rows c0 .. c0+63
+                float* base = p.dq_acc + (static_cast<size_t>(bhq) * p.N + static_cast<size_t>(i) * kTileM) * D + r;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t v32[32];
+                    tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, v32);
+                    tmem_ld_wait();
+                    const int qbase = i * kTileM + c0 + h * 32;
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if (qbase + t < p.N)
+                            red_add_f32(base + static_cast<size_t>(c0 + h * 32 + t) * D, __uint_as_float(v32[t]));
+                }
+            } else {
+                // lanes = query rows, columns = head dim; this half takes columns wg*32 .. +31
+                const int qrow = i * kTileM + r;
+                uint32_t v32[32];
+                tmem_ld32(tmem + lane_off + kColDP + wg * 32, v32);
+                tmem_ld_wait();
+                if (qrow < p.N) {
+                    float* dst = p.dq_acc + (static_cast<size_t>(bhq) * p.N + qrow) * D + wg * 32;
+#pragma unroll
+                    for (int t = 0; t < 8; ++t)
+                        red_add_v4(dst + 4 * t, __uint_as_float(v32[4 * t]), __uint_as_float(v32[4 * t + 1]),
+                                   __uint_as_float(v32[4 * t + 2]), __uint_as_float(v32[4 * t + 3]));
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(dq_free);
+            return true;
+        };
+
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
+            const int st = it & 1;
             const uint32_t ph = it & 1;
             const int g = it / per_head;
             const int i = i0 + (it - g * per_head);
-            ok = mbar_wait(q_full, ph, abort_flag, kBSiteQ) && mbar_wait(s_full, ph, abort_flag, kBSiteS);
+            const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
+            const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
+            // ---- P^T = 2^(S^T c - lse2)
+            ok = mbar_wait(&q_full[st], (it >> 1) & 1, abort_flag, kBSiteQ) && mbar_wait(s_full, ph, abort_flag, kBSiteS);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-            uint32_t sr[4][32];
+            {
+                uint32_t sr[2][32];
+                tmem_ld32(tmem + lane_off + kColS + c0, sr[0]);
+                tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
+                tmem_ld_wait();
+                const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                const bool diag = p.causal && (i == j);
 #pragma unroll
-            for (int q = 0; q < 4; ++q) tmem_ld32(tmem + lane_off + kColS + q * 32, sr[q]);
-            tmem_ld_wait();
-            float* pv = reinterpret_cast<float*>(&sr[0][0]);
-            const bool diag = p.causal && (i == j);
-            const bool kv_ok = kv < p.N;
+                for (int q = 0; q < 64; ++q) {
+                    float e = ex2(fmaf(sv[q], c, -lse_s[q]));
+                    if (!kv_ok || (diag && c0 + q < r)) e = 0.f;
+                    pv[q] = e;
+                }
+                uint32_t pk[32];
 #pragma unroll
-            for (int q = 0; q < 128; ++q) {
-                float e = ex2(fmaf(pv[q], c, -lse_s[q]));
-                if (!kv_ok || (diag && q < r)) e = 0.f;
-                pv[q] = e;
+                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(pv[2 * t], pv[2 * t + 1]);
+                tmem_st32(tmem + lane_off + kColS + wg * 32, pk);
+                tmem_st_wait();
             }
-            uint32_t pk[64];
-#pragma unroll
-            for (int t = 0; t < 64; ++t) pk[t] = pack_bf16x2(pv[2 * t], pv[2 * t + 1]);
-            tmem_st32(tmem + lane_off + kColS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tmem + lane_off + kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-            tmem_st_wait();
             tc_fence_before();
             mbar_arrive(p_full);
-            // dS^T = P^T o (dP^T - D) * scale  -> shared memory (K-major, 128B swizzle)
-            ok = (it == 0 || mbar_wait(ds_empty, ph ^ 1, abort_flag, kBSiteDSEmpty)) &&
-                 mbar_wait(dp_full, ph, abort_flag, kBSiteDP);
+            // ---- previous dQ tile out of tensor memory
+            if (it > 0) {
+                ok = drain_dq(it - 1);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            }
+            // ---- dS^T = P^T o (dP^T - D) * scale  -> shared memory (K-major, 128B swizzle)
+            ok = mbar_wait(dp_full, ph, abort_flag, kBSiteDP);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+            for (int h = 0; h < 2; ++h) {
                 uint32_t dpr[32];
-                tmem_ld32(tmem + lane_off + kColDP + q4 * 32, dpr);
+                tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
                 tmem_ld_wait();
                 uint32_t w[16];
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
-                    const int q0 = q4 * 32 + 2 * t;
+                    const int q0 = h * 32 + 2 * t;
                     const float d0 = pv[q0] * (__uint_as_float(dpr[2 * t]) - dvec_s[q0]) * p.scale;
                     const float d1 = pv[q0 + 1] * (__uint_as_float(dpr[2 * t + 1]) - dvec_s[q0 + 1]) * p.scale;
                     w[t] = pack_bf16x2(d0, d1);
                 }
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    const uint32_t off = sw128_offset(r, q4 * 32 + v * 8, kTileN);
+                    const uint32_t off = sw128_offset(r, c0 + h * 32 + v * 8, kTileN);
                     *reinterpret_cast<uint4*>(ds_s + off) = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
                 }
             }
@@ -379,19 +494,24 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_before();
             mbar_arrive(ds_full);
         }
+        if (ok && n_it > 0) {
+            ok = drain_dq(n_it - 1);
+            ok = __all_sync(0xffffffffu, ok);
+        }
         // ---- epilogue: dV, dK rows of this key block (summed over the group)
         if (ok && n_it > 0) {
             ok = mbar_wait(dkv_full, 0, abort_flag, kBSiteDKV);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                const bool valid = kv < p.N;
                 const size_t row = static_cast<size_t>(bkv) * p.N + kv;
+                constexpr int kHalf = D / 2;  // columns of dK/dV written by this warp group
 #pragma unroll 1
                 for (int which = 0; which < 2; ++which) {
-                    const uint32_t col0 = which == 0 ? kColDV : kColDK;
-                    __nv_bfloat16* dst_row = reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D;
+                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kHalf;
+                    __nv_bfloat16* dst_row =
+                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kHalf;
 #pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
+                    for (int q = 0; q < kHalf / 32; ++q) {
                         uint32_t v32[32];
                         tmem_ld32(tmem + lane_off + col0 + q * 32, v32);
                         tmem_ld_wait();
@@ -399,7 +519,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                         for (int t = 0; t < 16; ++t)
                             pk[t] = pack_bf16x2(__uint_as_float(v32[2 * t]), __uint_as_float(v32[2 * t + 1]));
-                        if (valid) {
+                        if (kv_ok) {
                             uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
 #pragma unroll
                             for (int t = 0; t < 4; ++t)
@@ -408,36 +528,6 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                 }
             }
-        }
-    } else {
-        // ------------------------------------------------------------ dQ drain
-        const int wq = warp - 4;
-        const int r = (wq << 5) + lane;  // query row inside the tile = TMEM lane
-        const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
-        for (int it = 0; it < n_it; ++it) {
-            const int g = it / per_head;
-            const int i = i0 + (it - g * per_head);
-            const int bhq = b * p.Hq + hkv * G + g;
-            bool ok = mbar_wait(dq_full, it & 1, abort_flag, kBSiteDQ);
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            const int qrow = i * kTileM + r;
-            float* dst = p.dq_acc + (static_cast<size_t>(bhq) * p.N + qrow) * D;
-#pragma unroll 1
-            for (int q = 0; q < D / 32; ++q) {
-                uint32_t v32[32];
-                tmem_ld32(tmem + lane_off + kColDP + q * 32, v32);
-                tmem_ld_wait();
-                if (qrow < p.N) {
-#pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        atomicAdd(reinterpret_cast<float4*>(dst + q * 32 + 4 * t),
-                                  make_float4(__uint_as_float(v32[4 * t]), __uint_as_float(v32[4 * t + 1]),
-                                              __uint_as_float(v32[4 * t + 2]), __uint_as_float(v32[4 * t + 3])));
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(dq_free);
         }
     }
 

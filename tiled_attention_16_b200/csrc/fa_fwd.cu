@@ -93,10 +93,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: heaviest (last) query blocks first for causal balance
+    // ---- work unit: head groups; inside a group the heaviest (last) query
+    //      blocks come first for causal balance, then the head
     const int BH = p.B * p.Hq;
-    const int mb = p.n_mblocks - 1 - static_cast<int>(blockIdx.x) / BH;
-    const int bh = static_cast<int>(blockIdx.x) % BH;
+    const int tile = static_cast<int>(blockIdx.x);
+    const int grp = tile / (p.heads_per_group * p.n_mblocks);
+    const int h_first = grp * p.heads_per_group;
+    const int nh = min(p.heads_per_group, BH - h_first);
+    const int rr = tile - grp * p.heads_per_group * p.n_mblocks;
+    const int mb = p.n_mblocks - 1 - rr / nh;
+    const int bh = h_first + rr % nh;
     const int b = bh / p.Hq;
     const int h = bh - b * p.Hq;
     const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);

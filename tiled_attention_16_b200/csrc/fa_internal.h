@@ -11,11 +11,16 @@ namespace fa {
 constexpr int kTileM = 128;  // query rows per MMA tile (TMEM lanes)
 constexpr int kTileN = 128;  // key/value rows per tile
 
+// Work-unit order: units are taken head group by head group (heads_per_group
+// consecutive (batch, head) pairs), heaviest causal block first inside a
+// group, so the K/V (forward) or Q/dO/dQ (backward) working set of the CTAs
+// resident at one time stays inside the 126 MB L2.
 struct FwdParams {
     int B, Hq, Hkv, N;
     int causal;
     float scale_log2;  // softmax scale * log2(e)
     int n_mblocks;     // ceil(N / 256): work unit = two 128-row query tiles
+    int heads_per_group;
     void* o;           // bf16 [B,Hq,N,D]
     float* lse;        // fp32 [B,Hq,N]
 };
@@ -23,6 +28,7 @@ struct FwdParams {
 struct BwdParams {
     int B, Hq, Hkv, N, Npad;
     int causal;
+    int heads_per_group;  // K/V heads per scheduling group
     float scale;       // softmax scale (dS is pre-multiplied by it)
     float scale_log2;  // scale * log2(e)
     const float* lse2; // [B*Hq, Npad] lse * log2(e), +inf on padding rows
