@@ -193,6 +193,28 @@ def config_of(wl, ws):
             "parallelism": f"{ws} independent replica(s), one per GPU"}
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(wl, rank: int):
+    """Each rank solves its own independent problem of the same size."""
+    return wl.with_(seed=wl.seed + rank)
+
+
+def max_over_ranks(ms: float, ws: int, device) -> float:
+    """Slowest rank's elapsed time (the job time of independent replicas)."""
+    if ws <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step: float, ws: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank's flops over the max-over-ranks step time."""
+    return flops_per_step * ws / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_gpu(args, wl):
     import torch
@@ -214,7 +236,7 @@ def run_gpu(args, wl):
     torch.cuda.set_device(dev)
 
     # inputs resident in HBM (rank r draws its own problem: seed + r)
-    q, k, v, do = (x.to(dev) for x in make_inputs(wl.with_(seed=wl.seed + rank)))
+    q, k, v, do = (x.to(dev) for x in make_inputs(rank_workload(wl, rank)))
     o = torch.empty_like(q)
     lse = torch.empty((wl.B, wl.Hq, wl.N), device=dev, dtype=torch.float32)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -250,14 +272,10 @@ def run_gpu(args, wl):
     clocks = sampler.stop()
     if A.device_status(dev) != A.FA_OK:
         raise RuntimeError(f"device status not OK after timing (sites {A.timeout_sites():#x})")
-    ms_total = e0.elapsed_time(e1)
-    if ws > 1:
-        t = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(e0.elapsed_time(e1), ws, dev)
     ms = ms_total / args.steps
     flops_step = wl.flops_fwd() + wl.flops_bwd()
-    value = flops_step * ws / (ms * 1e-3) / 1e12
+    value = job_tflops(flops_step, ws, ms)
 
     # kernel-level numbers from the live events
     kms = {k: (t / n if n else None) for k, (t, n) in per_kernel.items()}
@@ -292,7 +310,7 @@ def run_gpu(args, wl):
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (x.pin_memory() for x in make_inputs(wl.with_(seed=wl.seed + rank)))
+        hq, hk, hv, hdo = (x.pin_memory() for x in make_inputs(rank_workload(wl, rank)))
         ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
         hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
         hdq = torch.empty(dq.shape, dtype=dq.dtype, pin_memory=True)
@@ -325,12 +343,8 @@ def run_gpu(args, wl):
             e2e_step()
         a1.record(stream)
         torch.cuda.synchronize()
-        e_ms = a0.elapsed_time(a1)
-        if ws > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": flops_step * ws / (e_ms / e2e_steps * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(a0.elapsed_time(a1), ws, dev)
+        e2e = {"value": job_tflops(flops_step, ws, e_ms / e2e_steps), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
 
     cpu = None
