@@ -57,7 +57,8 @@ typedef enum {
     FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad sizes, bad scale, small workspace */
     FA_ERR_UNSUPPORTED = 2, /* head dimension other than 64 or 128, or a non-sm_100 device */
     FA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
-    FA_ERR_TIMEOUT = 4      /* a device-side pipeline wait gave up (reported by fa_get_device_status) */
+    FA_ERR_TIMEOUT = 4,     /* a device-side pipeline wait gave up (reported by fa_get_device_status) */
+    FA_ERR_TOO_LARGE = 5    /* fa_bwd_noalloc: the shape needs more than FA_NOALLOC_SCRATCH_BYTES */
 } fa_status;
 
 /* Problem shape.  Hkv == Hq is plain multi-head attention; Hkv < Hq is GQA
@@ -87,6 +88,33 @@ FA_API fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, con
                  const void* o, const void* dout, const float* lse,
                  void* dq, void* dk, void* dv,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward that allocates nothing (the pages have no counterpart: this is a
+ * deployment convenience, not part of the method).
+ *
+ * Same computation, arguments and outputs as fa_bwd, but without a caller
+ * workspace: the scratch it needs (the per-row LSE/D statistics and the fp32
+ * dQ accumulator, fa_bwd_workspace_bytes(shape) bytes) lives in a fixed
+ * FA_NOALLOC_SCRATCH_BYTES region of device memory that the library reserves
+ * statically on every GPU that loads it, held until the process exits.  It is
+ * meant for callers that cannot call cudaMalloc or hand out device memory on
+ * this path: plugins whose host runtime owns every device allocation, or
+ * latency-bound code where an allocation (and the synchronisation it can
+ * imply) is not acceptable.
+ *   - Shapes whose scratch exceeds FA_NOALLOC_SCRATCH_BYTES are rejected with
+ *     FA_ERR_TOO_LARGE before anything is launched (use fa_bwd for those).
+ *   - The first call on a device looks up the region's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - Every call on a device shares the one region, and each call re-zeroes
+ *     the parts that must start at zero; calls that overlap on the GPU (other
+ *     streams, other host threads) race on it and must be serialised by the
+ *     caller.
+ *   - No cudaMalloc, cudaFree or allocating library routine is called. */
+#define FA_NOALLOC_SCRATCH_BYTES (32u << 20)
+FA_API fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, const void* v,
+                                const void* o, const void* dout, const float* lse,
+                                void* dq, void* dk, void* dv, void* stream);
 
 /* Synchronises `stream`, then reports and clears the device status word of
  * the current device: FA_ERR_TIMEOUT if any kernel gave up a bounded wait

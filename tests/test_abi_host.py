@@ -18,14 +18,15 @@ build()
 def test_exports_every_declared_symbol():
     names = A.declared_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
-                          "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end"}
+                          "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
+                          "fa_bwd_noalloc"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
 
 
 def test_status_strings():
-    for s in range(5):
+    for s in range(6):
         assert isinstance(A.status_str(s), str) and A.status_str(s)
     assert A.status_str(99) == "unknown status"
 
@@ -124,3 +125,20 @@ def test_profile_hooks_without_launches():
     assert set(res) == set(A.PROFILE_KINDS)
     assert all(v == (0.0, 0) for v in res.values())
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
+
+
+def _noalloc(shape, ptr=P, **over):
+    args = {n: ptr for n in ("q", "k", "v", "o", "do", "lse", "dq", "dk", "dv")}
+    args.update(over)
+    return A.lib().fa_bwd_noalloc(None if shape is None else ctypes.byref(shape), args["q"], args["k"], args["v"],
+                                  args["o"], args["do"], args["lse"], args["dq"], args["dk"], args["dv"], None)
+
+
+def test_noalloc_host_checks():
+    assert _noalloc(None) == A.FA_ERR_INVALID_ARG
+    assert _noalloc(shape(N=0)) == A.FA_ERR_INVALID_ARG
+    assert _noalloc(shape(D=96)) == A.FA_ERR_UNSUPPORTED
+    assert _noalloc(shape(), dq=P + 8) == A.FA_ERR_INVALID_ARG
+    big = A.make_shape(1, 32, 32, 4096, 128, 0.1, 1)
+    assert A.lib().fa_bwd_workspace_bytes(ctypes.byref(big)) > A.NOALLOC_SCRATCH_BYTES
+    assert _noalloc(big) == A.FA_ERR_TOO_LARGE

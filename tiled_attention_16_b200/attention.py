@@ -19,7 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libfa_sm100.so")
 HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "fa.h")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_TOO_LARGE = range(6)
+NOALLOC_SCRATCH_BYTES = 32 << 20  # FA_NOALLOC_SCRATCH_BYTES in include/fa.h
 
 
 class FaShape(ctypes.Structure):
@@ -58,6 +59,8 @@ def lib() -> ctypes.CDLL:
         L.fa_status_str.restype = ctypes.c_char_p
         L.fa_debug_timeout_sites.argtypes = []
         L.fa_debug_timeout_sites.restype = ctypes.c_uint
+        L.fa_bwd_noalloc.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.fa_bwd_noalloc.restype = ctypes.c_int
         L.fa_profile_begin.argtypes = []
         L.fa_profile_begin.restype = ctypes.c_int
         L.fa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
@@ -160,6 +163,32 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
                       workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None, dq=None, dk=None, dv=None):
+    """Backward through fa_bwd_noalloc: no workspace argument, the library's
+    static scratch is used (for callers that must not allocate device memory
+    on this path).  Output tensors may be passed in to avoid allocating them
+    here too.  Calls on one device share the scratch, so they must not overlap."""
+    B, Hq, Hkv, N, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    for t, name, shape in ((q, "q", (B, Hq, N, D)), (k, "k", (B, Hkv, N, D)), (v, "v", (B, Hkv, N, D)),
+                           (o, "o", (B, Hq, N, D)), (do, "do", (B, Hq, N, D))):
+        _check(t, name, shape)
+    _check(lse, "lse", (B, Hq, N), torch.float32)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", (B, Hq, N, D))
+    _check(dk, "dk", (B, Hkv, N, D))
+    _check(dv, "dv", (B, Hkv, N, D))
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    st = lib().fa_bwd_noalloc(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                              _stream_ptr(q.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -82,6 +82,29 @@ fa_status check_device() {
 
 unsigned int g_last_sites = 0;
 
+// Scratch of fa_bwd_noalloc: reserved statically in device memory on every
+// GPU that loads the library, so that entry point never allocates.  In host
+// code this name only stands in for the symbol; the device address comes from
+// cudaGetSymbolAddress (noalloc_scratch below).
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+fa_status noalloc_scratch(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    static std::mutex mu;
+    static void* cache[64] = {};
+    std::lock_guard<std::mutex> g(mu);
+    if (cache[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+        cache[dev] = ptr;
+    }
+    *out = cache[dev];
+    return FA_OK;
+}
+
 // ---- optional per-kernel event timing (fa_profile_begin / fa_profile_end)
 struct Profiler {
     std::mutex mu;
@@ -140,6 +163,7 @@ const char* fa_status_str(fa_status s) {
         case FA_ERR_UNSUPPORTED: return "unsupported (head dim or device)";
         case FA_ERR_CUDA: return "CUDA error";
         case FA_ERR_TIMEOUT: return "device-side wait timed out";
+        case FA_ERR_TOO_LARGE: return "problem needs more scratch than the library's static region";
     }
     return "unknown status";
 }
@@ -234,6 +258,23 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
             return launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
         });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// fa_bwd with its workspace taken from the library's static scratch instead of
+// the caller: for callers that cannot allocate device memory on this path.
+fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, void* stream) {
+    fa_status st = check_shape(shape);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+        return FA_ERR_INVALID_ARG;
+    if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D).total > FA_NOALLOC_SCRATCH_BYTES)
+        return FA_ERR_TOO_LARGE;
+    if ((st = check_device()) != FA_OK) return st;
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != FA_OK) return st;
+    return fa_bwd(shape, q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 fa_status fa_get_device_status(void* stream) {
