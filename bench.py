@@ -283,25 +283,30 @@ def run_gpu(args, wl):
     bwd_ms = sum(x for k, x in kms.items() if k != "fa_fwd_kernel" and x)
     peaks, peak_src = load_peaks()
     peak_tf = peaks["bf16_tflops"]
-    bwd_main = kms["fa_bwd_kernel"]
-    # the main backward kernel performs all five backward GEMMs
-    achieved = wl.flops_bwd() / (bwd_main * 1e-3) / 1e12
-    dominant = max(kms, key=lambda k: kms[k] or 0)
-    roofline = {"kernel": "fa_bwd_kernel", "bound": "tensor", "achieved": achieved, "peak": peak_tf,
-                "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": recorded_traffic("fa_bwd_kernel", wl.name),
-                "peak_source": f"{peak_src} bf16_tflops (burst)", "dominant_by_time": dominant,
-                "per_launch_ms": bwd_main}
+    # GEMM flops each tensor kernel executes (one "GEMM" over a head = 2*N^2*D,
+    # halved when causal): fused backward 5, dK/dV kernel 4 (S, dP, dV, dK),
+    # dQ kernel 3 (S and dP recomputed, dQ).
+    gemm = wl.flops_fwd() / 2
+    kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
+                    "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm}
+    tensor_k = {k: v for k, v in kms.items() if v and k in kernel_flops}
+    dominant = max(tensor_k, key=lambda k: tensor_k[k])
+    achieved = kernel_flops[dominant] / (tensor_k[dominant] * 1e-3) / 1e12
+    roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": recorded_traffic(dominant, wl.name),
+                "peak_source": f"{peak_src} bf16_tflops (burst)", "per_launch_ms": tensor_k[dominant],
+                "flops_per_launch": kernel_flops[dominant]}
     fwd_tf = wl.flops_fwd() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = wl.flops_bwd() / (bwd_ms * 1e-3) / 1e12
-    pre_bytes = wl.B * wl.Hq * wl.N * (2 * wl.D * 2 + 4 + 8) + wl.B * wl.Hq * wl.N * wl.D * 4
+    pre_zero = wl.B * wl.Hq * wl.N * wl.D * 4 if kms.get("fa_bwd_kernel") else 0
+    pre_bytes = wl.B * wl.Hq * wl.N * (2 * wl.D * 2 + 4 + 8) + pre_zero
     conv_bytes = wl.B * wl.Hq * wl.N * wl.D * (4 + 2)
     breakdown = {
         "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_of_peak": fwd_tf / peak_tf,
         "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_of_peak": bwd_tf / peak_tf,
-        "bwd_main_ms": bwd_main,
-        "bwd_preprocess_ms": kms["fa_bwd_preprocess"],
+        "bwd_mode": "separate dQ pass" if kms.get("fa_bwd_dq_kernel") else "fused (fp32 dQ reductions)",
+        "bwd_kernels_ms": {k: v for k, v in kms.items() if v and k != "fa_fwd_kernel"},
         "bwd_preprocess_gbs": pre_bytes / (kms["fa_bwd_preprocess"] * 1e-3) / 1e9 if kms["fa_bwd_preprocess"] else None,
-        "bwd_dq_convert_ms": kms["fa_bwd_dq_convert"],
         "bwd_dq_convert_gbs": conv_bytes / (kms["fa_bwd_dq_convert"] * 1e-3) / 1e9 if kms["fa_bwd_dq_convert"] else None,
         "hbm_peak_gbs": peaks["hbm_gbs"],
     }

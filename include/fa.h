@@ -134,9 +134,12 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * launching stream.  fa_profile_end() waits for those events, writes for each
  * kernel kind k the summed duration total_ms[k] and the launch count
  * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
- * preprocess, 2 backward main, 3 backward dQ convert (FA_PROFILE_KINDS).
- * Events are host-created objects; no device memory is allocated. */
-#define FA_PROFILE_KINDS 4
+ * preprocess, 2 fused backward (dK, dV and dQ by fp32 reductions), 3 dQ
+ * convert, 4 backward dK/dV kernel, 5 backward dQ kernel (FA_PROFILE_KINDS;
+ * fa_bwd uses 1, 4, 5 by default and 1, 2, 3 when the environment variable
+ * FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
+ * objects; no device memory is allocated. */
+#define FA_PROFILE_KINDS 6
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

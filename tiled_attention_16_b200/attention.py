@@ -202,7 +202,8 @@ def timeout_sites() -> int:
     return int(lib().fa_debug_timeout_sites())
 
 
-PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert")
+PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
+                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel")
 
 
 def profile_begin() -> None:
@@ -213,8 +214,8 @@ def profile_begin() -> None:
 
 def profile_end() -> dict:
     """{kernel name: (total ms, launches)} for the launches since profile_begin()."""
-    ms = (ctypes.c_float * 4)()
-    n = (ctypes.c_int * 4)()
+    ms = (ctypes.c_float * len(PROFILE_KINDS))()
+    n = (ctypes.c_int * len(PROFILE_KINDS))()
     st = lib().fa_profile_end(ms, n)
     if st != FA_OK:
         raise FAError(st, "fa_profile_end")

@@ -5,6 +5,7 @@
 #include "fa_internal.h"
 
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -81,6 +82,21 @@ fa_status check_device() {
 }
 
 unsigned int g_last_sites = 0;
+
+constexpr int kNumSMs = 148;
+
+// dQ strategy of the backward: a separate dQ pass (default; deterministic, no
+// reductions) or the fused kernel with fp32 reductions ("atomic").  Chosen by
+// measurement; FA_DQ_MODE=atomic|separate overrides it (read once).
+bool dq_separate_mode() {
+    static int mode = -1;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = std::getenv("FA_DQ_MODE");
+        mode = (e && std::strcmp(e, "atomic") == 0) ? 0 : 1;
+    });
+    return mode == 1;
+}
 
 // Scratch of fa_bwd_noalloc: reserved statically in device memory on every
 // GPU that loads the library, so that entry point never allocates.  In host
@@ -232,31 +248,48 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.N = s.N;
     p.Npad = Npad;
     p.causal = s.causal ? 1 : 0;
-    // K/V heads per scheduling group: keep the group's Q, dO (bf16) and dQ
-    // accumulator (fp32) of all its query heads within ~48 MiB of L2.
+    const bool separate = dq_separate_mode();
+    const int T = (s.N + kTileM - 1) / kTileM;
+    // K/V heads per scheduling group of the key-block kernels: keep the
+    // group's Q, dO (bf16) and, for the fused kernel, the fp32 dQ accumulator
+    // of all its query heads within ~48 MiB of L2.  With fewer than two waves
+    // of work units, one group (global heaviest-first order) balances better.
     {
-        const double per_kv_head = 8.0 * s.N * s.D * (s.Hq / s.Hkv);
-        const int g = static_cast<int>(48.0 * 1024 * 1024 / per_kv_head);
+        const double per_kv_head = (separate ? 4.0 : 8.0) * s.N * s.D * (s.Hq / s.Hkv);
+        int g = static_cast<int>(48.0 * 1024 * 1024 / per_kv_head);
+        if (static_cast<long long>(T) * s.B * s.Hkv < 2LL * kNumSMs) g = s.B * s.Hkv;
         p.heads_per_group = g < 1 ? 1 : (g > s.B * s.Hkv ? s.B * s.Hkv : g);
+    }
+    // query heads per group of the dQ pass: K/V streamed by the group in ~32 MiB
+    {
+        const double per_head = 4.0 * s.N * s.D / (s.Hq / s.Hkv);
+        const int g = static_cast<int>(32.0 * 1024 * 1024 / per_head);
+        p.dq_heads_per_group = g < 1 ? 1 : (g > s.B * s.Hq ? s.B * s.Hq : g);
     }
     p.scale = s.scale;
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
-    p.lse2 =reinterpret_cast<const float*>(wsb + ws.lse2_off);
+    p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2_off);
     p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec_off);
     p.dq_acc = reinterpret_cast<float*>(wsb + ws.dq_off);
+    p.dq = dq;
     p.dk = dk;
     p.dv = dv;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(1, strm, [&] {
         return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
-                                     reinterpret_cast<float*>(wsb + ws.dvec_off), p.dq_acc, s.B * s.Hq, s.N, Npad,
-                                     strm);
+                                     reinterpret_cast<float*>(wsb + ws.dvec_off), separate ? nullptr : p.dq_acc,
+                                     s.B * s.Hq, s.N, Npad, s.scale, strm);
     });
-    if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
-    if (e == cudaSuccess)
-        e = timed(3, strm, [&] {
-            return launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
-        });
+    if (separate) {
+        if (e == cudaSuccess) e = timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });
+        if (e == cudaSuccess) e = timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
+    } else {
+        if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
+        if (e == cudaSuccess)
+            e = timed(3, strm, [&] {
+                return launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
+            });
+    }
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

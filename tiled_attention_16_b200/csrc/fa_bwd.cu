@@ -9,7 +9,7 @@
 // 改进2 parallelises the sequence dimension).
 //
 // Three launches:
-//   1. fa_bwd_preprocess: D_i = sum_d dO_id O_id and lse2_i = lse_i*log2(e)
+//   1. fa_bwd_preprocess: scale * D_i (D_i = sum_d dO_id O_id) and lse2_i = lse_i*log2(e)
 //      (both padded to a multiple of 128 rows: D = 0, lse2 = +inf, so padded
 //      query rows get P = 0), and zeroes the fp32 dQ accumulator.  HBM-bound.
 //   2. fa_bwd_kernel: one CTA per (batch, K/V head, 128-row key block j).
@@ -31,7 +31,8 @@
 //              end they write dK and dV.
 //   warp  8    MMA issuer (one thread)
 //   warp  9    TMA producer
-// Tensor memory: S^T (P^T over its first half) | dP^T, then dQ | dV | dK.
+// Tensor memory: S^T (P^T packed over the columns each compute group read) |
+// dP^T, then dQ | dV | dK.
 // MMA issue order per query tile it:
 //   S(it) ; dK(it-1), dQ(it-1) ; dP(it) ; dV(it)
 // so the tensor core works on S and dK/dQ while the compute warps form P and
@@ -88,6 +89,12 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     }
 }
 
+// TMEM column (relative to the S^T block) of K-step kk (16 query rows) of the
+// packed bf16 P^T: query columns 0-63 are packed into columns 0-31 and query
+// columns 64-127 into columns 64-95, i.e. each compute group overwrites only
+// fp32 S^T columns it has already read itself.
+__host__ __device__ constexpr uint32_t p_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
+
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
     asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
 }
@@ -103,7 +110,7 @@ template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                   const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
-                  float4* __restrict__ dq_acc, size_t dq_vec4, int BH, int N, int Npad) {
+                  float4* __restrict__ dq_acc, size_t dq_vec4, int BH, int N, int Npad, float scale) {
     constexpr int kPer = D / 32;  // elements per lane
     const int lane = threadIdx.x & 31;
     const size_t warp_id = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -138,7 +145,7 @@ fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __re
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) {
-            dvec[row] = acc;
+            dvec[row] = acc * scale;  // the backward kernels use scale * D
             lse2[row] = (n < N) ? lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f : INFINITY;
         }
     }
@@ -362,7 +369,7 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tc_fence_after();
 #pragma unroll
                 for (int kk = 0; kk < kTileM / 16; ++kk)
-                    mma_ts(tmem + kColDV, tmem + kColS + kk * 8, sdesc_sw128(da + kk * 2048, kAtom, 1024), kIdAcc,
+                    mma_ts(tmem + kColDV, tmem + kColS + p_col(kk), sdesc_sw128(da + kk * 2048, kAtom, 1024), kIdAcc,
                            (it > 0 || kk > 0));
                 tc_commit(&do_empty[st]);
             }
@@ -447,17 +454,27 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
                 tmem_ld_wait();
                 const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                // masked only on the diagonal / partial last key block (warp-uniform test);
+                // there, query columns q < lo are zero
                 const bool diag = p.causal && (i == j);
-#pragma unroll
-                for (int q = 0; q < 64; ++q) {
-                    float e = ex2(fmaf(sv[q], c, -lse_s[q]));
-                    if (!kv_ok || (diag && c0 + q < r)) e = 0.f;
-                    pv[q] = e;
+                if (diag || (j + 1) * kTileN > p.N) {
+                    const int lo = !kv_ok ? 64 : (diag ? r - c0 : 0);
+                    static_for<0, 64>([&](auto qc) {
+                        constexpr int q = decltype(qc)::value;
+                        const float e = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
+                        pv[q] = (q >= lo) ? e : 0.f;
+                    });
+                } else {
+                    static_for<0, 64>([&](auto qc) {
+                        constexpr int q = decltype(qc)::value;
+                        pv[q] = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
+                    });
                 }
                 uint32_t pk[32];
 #pragma unroll
                 for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(pv[2 * t], pv[2 * t + 1]);
-                tmem_st32(tmem + lane_off + kColS + wg * 32, pk);
+                // each group packs its P^T half into the columns it has just read
+                tmem_st32(tmem + lane_off + kColS + c0, pk);
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -479,9 +496,10 @@ fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 uint32_t w[16];
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
+                    // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
                     const int q0 = h * 32 + 2 * t;
-                    const float d0 = pv[q0] * (__uint_as_float(dpr[2 * t]) - dvec_s[q0]) * p.scale;
-                    const float d1 = pv[q0 + 1] * (__uint_as_float(dpr[2 * t + 1]) - dvec_s[q0 + 1]) * p.scale;
+                    const float d0 = pv[q0] * fmaf(__uint_as_float(dpr[2 * t]), p.scale, -dvec_s[q0]);
+                    const float d1 = pv[q0 + 1] * fmaf(__uint_as_float(dpr[2 * t + 1]), p.scale, -dvec_s[q0 + 1]);
                     w[t] = pack_bf16x2(d0, d1);
                 }
 #pragma unroll
@@ -562,18 +580,18 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D) {
 }
 
 cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse, float* lse2, float* dvec,
-                                  float* dq_acc, int BH, int N, int Npad, cudaStream_t stream) {
+                                  float* dq_acc, int BH, int N, int Npad, float scale, cudaStream_t stream) {
     const size_t rows = static_cast<size_t>(BH) * Npad;
-    const size_t dq_vec4 = static_cast<size_t>(BH) * N * D / 4;
+    const size_t dq_vec4 = dq_acc ? static_cast<size_t>(BH) * N * D / 4 : 0;
     const int grid = grid_for(rows * 32 > dq_vec4 ? rows * 32 : dq_vec4, 256);
     if (D == 128)
         fa_bwd_preprocess<128><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                          static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec,
-                                                         reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad);
+                                                         reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale);
     else
         fa_bwd_preprocess<64><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                         static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec,
-                                                        reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad);
+                                                        reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale);
     return cudaGetLastError();
 }
 

@@ -1,0 +1,716 @@
+// fa_bwd_split.cu — tiled attention backward with a separate dQ pass.
+//
+// Same mathematics as fa_bwd.cu (recompute P from the saved LSE, closed-form
+// softmax gradient dS = P o (dP - D); "FlashAttention V2深度解析：反向传播显存
+// 优化让大模型训练不再OOM", sections 改进1 and 改进2), split into two kernels
+// so that no fp32 reduction into global memory is needed and the result is
+// deterministic:
+//
+//   fa_bwd_dkdv_kernel  one CTA per (batch, K/V head, 128-row key block j);
+//                       loops over the query heads of the GQA group and the
+//                       query tiles i (i >= j when causal):
+//                         S^T = K_j Q_i^T, P^T = 2^(S^T c - lse2), dP^T = V_j dO_i^T,
+//                         dV += P^T dO_i, dS^T = P^T o (dP^T - D) * scale, dK += dS^T Q_i.
+//                       P^T and dS^T never leave tensor memory: each is packed
+//                       as bf16 over the fp32 columns it was computed from and
+//                       read from there as the A operand of the dV / dK MMA.
+//   fa_bwd_dq_kernel    one CTA per (batch, query head, 128-row query tile i);
+//                       loops over key tiles j (j <= i when causal):
+//                         S = Q_i K_j^T, P = 2^(S c - lse2), dP = dO_i V_j^T,
+//                         dS = P o (dP - D) * scale, dQ += dS K_j  (dQ in TMEM),
+//                       then writes dQ as bf16 once.
+//
+// The dQ pass recomputes S and dP (7 GEMMs per tile pair instead of 5), in
+// exchange for no reduction traffic and no serialisation on it.
+//
+// Both kernels: 320 threads = warps 0-7 compute (two groups of 4 warps split
+// the 128 columns of the score tile; thread = TMEM lane), warp 8 issues MMAs
+// (one thread), warp 9 drives TMA.  Every wait is bounded (sm100.cuh).
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
+
+namespace fa {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kCompute = 256;
+constexpr int kMaxDynSmem = 232448;
+
+// wait sites (bits of the device status word)
+enum SplitSite {
+    kS1Smem = 22, kS1Load = 23, kS1Empty = 24, kS1Mma = 25, kS1Compute = 26, kS1Drain = 27,
+    kS2Load = 28, kS2Mma = 29, kS2Compute = 30, kS2Drain = 31
+};
+
+// TMEM column (relative to a 128-column block) of K-step kk (16 columns of
+// the score tile) of a bf16 operand packed by the two compute groups: group g
+// packs its 64 columns into block columns [64g, 64g + 32).
+__host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
+
+__device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int site) {
+    if (mbar_try_wait(bar, parity)) return;
+    unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, 1u << site);
+            return;
+        }
+    }
+}
+
+template <int D>
+struct DkdvLayout {
+    static constexpr int kTileBytes = kTileM * D * 2;
+    static constexpr int kAtomBytes = kTileM * 128;
+    static constexpr int kK = 0;
+    static constexpr int kV = kK + kTileBytes;
+    static constexpr int kQ = kV + kTileBytes;       // 2 stages
+    static constexpr int kDO = kQ + 2 * kTileBytes;  // 2 stages
+    static constexpr int kLse = kDO + 2 * kTileBytes;
+    static constexpr int kDvec = kLse + 2 * kTileN * 4;
+    static constexpr int kBar = kDvec + 2 * kTileN * 4;
+    static constexpr int kNumBars = 16;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
+    static_assert(kBytes <= kMaxDynSmem, "dK/dV shared memory layout too large");
+};
+
+template <int D>
+struct DqLayout {
+    static constexpr int kTileBytes = kTileM * D * 2;
+    static constexpr int kAtomBytes = kTileM * 128;
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTileBytes;
+    static constexpr int kK = kDO + kTileBytes;      // 2 stages
+    static constexpr int kV = kK + 2 * kTileBytes;   // 2 stages
+    static constexpr int kBar = kV + 2 * kTileBytes;
+    static constexpr int kNumBars = 16;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
+    static_assert(kBytes <= kMaxDynSmem, "dQ shared memory layout too large");
+};
+
+// ===========================================================================
+// dK / dV
+// ===========================================================================
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                   const BwdParams p) {
+    using L = DkdvLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad + L::kBytes > static_cast<uint32_t>(L::kAlloc)) {
+        if (threadIdx.x == 0) atomicOr(&g_status, 1u << kS1Smem);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* kv_full = bars + 0;
+    uint64_t* q_full = bars + 1;    // [2]
+    uint64_t* q_empty = bars + 3;   // [2]
+    uint64_t* do_full = bars + 5;   // [2]
+    uint64_t* do_empty = bars + 7;  // [2]
+    uint64_t* s_full = bars + 9;
+    uint64_t* dp_full = bars + 10;
+    uint64_t* p_full = bars + 11;
+    uint64_t* ds_full = bars + 12;
+    uint64_t* dkv_full = bars + 13;
+    uint64_t* drain = bars + 14;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // work unit: head groups; inside a group key block j ascending (heaviest
+    // first when causal), then head
+    const int BHkv = p.B * p.Hkv;
+    const int T = (p.N + kTileM - 1) / kTileM;
+    const int tile = static_cast<int>(blockIdx.x);
+    const int grp = tile / (p.heads_per_group * T);
+    const int h0 = grp * p.heads_per_group;
+    const int nh = min(p.heads_per_group, BHkv - h0);
+    const int rr = tile - grp * p.heads_per_group * T;
+    const int j = rr / nh;
+    const int bkv = h0 + (rr - j * nh);
+    const int b = bkv / p.Hkv;
+    const int hkv = bkv - b * p.Hkv;
+    const int G = p.Hq / p.Hkv;
+    const int i0 = p.causal ? j : 0;
+    const int per_head = T - i0;
+    const int n_it = G * per_head;
+
+    if (threadIdx.x == 0) {
+        mbar_init(kv_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&do_full[s], 1);
+            mbar_init(&do_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(dp_full, 1);
+        mbar_init(p_full, kCompute);
+        mbar_init(ds_full, kCompute);
+        mbar_init(dkv_full, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+            for (int a = 0; a < D / 64; ++a) {
+                tma_load_3d(smem + L::kK + a * L::kAtomBytes, &tmK, kv_full, a * 64, j * kTileN, bkv);
+                tma_load_3d(smem + L::kV + a * L::kAtomBytes, &tmV, kv_full, a * 64, j * kTileN, bkv);
+            }
+            int issued_q = 0, issued_do = 0;
+            for (int it = 0; it < n_it; ++it) {
+                const int st = it & 1;
+                const int g = it / per_head;
+                const int i = i0 + (it - g * per_head);
+                const int bhq = b * p.Hq + hkv * G + g;
+                if (it >= 2 && !mbar_wait(&q_empty[st], ((it >> 1) - 1) & 1, abort_flag, kS1Empty)) break;
+                mbar_arrive_expect_tx(&q_full[st], L::kTileBytes + 2 * kTileM * 4);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kQ + st * L::kTileBytes + a * L::kAtomBytes, &tmQ, &q_full[st], a * 64,
+                                i * kTileM, bhq);
+                const size_t srow = static_cast<size_t>(bhq) * p.Npad + static_cast<size_t>(i) * kTileM;
+                bulk_load(smem + L::kLse + st * kTileM * 4, p.lse2 + srow, kTileM * 4, &q_full[st]);
+                bulk_load(smem + L::kDvec + st * kTileM * 4, p.dvec + srow, kTileM * 4, &q_full[st]);
+                issued_q = it + 1;
+                if (it >= 2 && !mbar_wait(&do_empty[st], ((it >> 1) - 1) & 1, abort_flag, kS1Empty)) break;
+                mbar_arrive_expect_tx(&do_full[st], L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kDO + st * L::kTileBytes + a * L::kAtomBytes, &tmDO, &do_full[st], a * 64,
+                                i * kTileM, bhq);
+                issued_do = it + 1;
+            }
+            wait_drain(kv_full, 0, kS1Drain);
+            for (int it = (issued_q > 2 ? issued_q - 2 : 0); it < issued_q; ++it)
+                wait_drain(&q_full[it & 1], (it >> 1) & 1, kS1Drain);
+            for (int it = (issued_do > 2 ? issued_do - 2 : 0); it < issued_do; ++it)
+                wait_drain(&do_full[it & 1], (it >> 1) & 1, kS1Drain);
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdSq = idesc_bf16_f32(kTileN, kTileM, 0, 0);  // S^T, dP^T
+            constexpr uint32_t kIdAcc = idesc_bf16_f32(kTileN, D, 0, 1);      // dV, dK (A from TMEM)
+            const uint32_t k_base = smem_u32(smem + L::kK);
+            const uint32_t v_base = smem_u32(smem + L::kV);
+            const uint32_t q_base = smem_u32(smem + L::kQ);
+            const uint32_t do_base = smem_u32(smem + L::kDO);
+            constexpr uint32_t kAtom = L::kAtomBytes;
+            auto issue_dk = [&](int itp) {
+                const uint32_t qa = q_base + (itp & 1) * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTileM / 16; ++kk)
+                    mma_ts(tmem + kColDK, tmem + kColDP + packed_col(kk), sdesc_sw128(qa + kk * 2048, kAtom, 1024),
+                           kIdAcc, (itp > 0 || kk > 0));
+                tc_commit(&q_empty[itp & 1]);
+            };
+            bool ok = mbar_wait(kv_full, 0, abort_flag, kS1Load);
+            for (int it = 0; ok && it < n_it; ++it) {
+                const int st = it & 1;
+                const uint32_t sph = (it >> 1) & 1;
+                const uint32_t ph = it & 1;
+                // S^T = K Q^T (the previous P^T was consumed by dV(it-1), issued earlier)
+                if (!(ok = mbar_wait(&q_full[st], sph, abort_flag, kS1Load))) break;
+                tc_fence_after();
+                const uint32_t qa = q_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    mma_ss(tmem + kColS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), kIdSq,
+                           kk > 0);
+                }
+                tc_commit(s_full);
+                // dK += dS^T Q of the previous query tile (dS^T packed in the dP^T block)
+                if (it > 0) {
+                    if (!(ok = mbar_wait(ds_full, ph ^ 1, abort_flag, kS1Mma))) break;
+                    tc_fence_after();
+                    issue_dk(it - 1);
+                }
+                // dP^T = V dO^T
+                if (!(ok = mbar_wait(&do_full[st], sph, abort_flag, kS1Load))) break;
+                tc_fence_after();
+                const uint32_t da = do_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    mma_ss(tmem + kColDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), kIdSq,
+                           kk > 0);
+                }
+                tc_commit(dp_full);
+                // dV += P^T dO
+                if (!(ok = mbar_wait(p_full, ph, abort_flag, kS1Mma))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int kk = 0; kk < kTileM / 16; ++kk)
+                    mma_ts(tmem + kColDV, tmem + kColS + packed_col(kk), sdesc_sw128(da + kk * 2048, kAtom, 1024),
+                           kIdAcc, (it > 0 || kk > 0));
+                tc_commit(&do_empty[st]);
+            }
+            if (ok && n_it > 0 && mbar_wait(ds_full, (n_it - 1) & 1, abort_flag, kS1Mma)) {
+                tc_fence_after();
+                issue_dk(n_it - 1);
+                tc_commit(dkv_full);
+            }
+            tc_commit(drain);
+            wait_drain(drain, 0, kS1Drain);
+        }
+    } else {
+        // ------------------------------------------------------------ compute (P^T, dS^T)
+        const int wg = warp >> 2;
+        const int wq = warp & 3;
+        const int r = (wq << 5) + lane;  // key row of the block = TMEM lane
+        const int kv = j * kTileN + r;
+        const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
+        const int c0 = wg * 64;          // this group's query columns
+        const float c = p.scale_log2;
+        const float sc = p.scale;
+        const bool kv_ok = kv < p.N;
+        const bool kv_block_partial = (j + 1) * kTileN > p.N;
+        float pv[64];
+        bool ok = true;
+        for (int it = 0; it < n_it; ++it) {
+            const int st = it & 1;
+            const uint32_t ph = it & 1;
+            const int g = it / per_head;
+            const int i = i0 + (it - g * per_head);
+            const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
+            const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
+            ok = mbar_wait(&q_full[st], (it >> 1) & 1, abort_flag, kS1Compute) &&
+                 mbar_wait(s_full, ph, abort_flag, kS1Compute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t sr[2][32];
+                tmem_ld32(tmem + lane_off + kColS + c0, sr[0]);
+                tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
+                tmem_ld_wait();
+                const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                // Masked only on the causal diagonal block and on a partial
+                // last key block (both uniform across the warp); there,
+                // columns q < lo are zero (lo = 64 masks a key row past N).
+                const bool diag = p.causal && (i == j);
+                if (diag || kv_block_partial) {
+                    const int lo = !kv_ok ? 64 : (diag ? r - c0 : 0);
+                    static_for<0, 64>([&](auto qc) {
+                        constexpr int q = decltype(qc)::value;
+                        const float e = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
+                        pv[q] = (q >= lo) ? e : 0.f;
+                    });
+                } else {
+                    static_for<0, 64>([&](auto qc) {
+                        constexpr int q = decltype(qc)::value;
+                        pv[q] = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
+                    });
+                }
+                uint32_t pk[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(pv[2 * t], pv[2 * t + 1]);
+                tmem_st32(tmem + lane_off + kColS + c0, pk);
+                tmem_st_wait();
+            }
+            tc_fence_before();
+            mbar_arrive(p_full);
+            ok = mbar_wait(dp_full, ph, abort_flag, kS1Compute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t dpr[32];
+                tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
+                    const int q0 = h * 32 + 2 * t;
+                    const float d0 = pv[q0] * fmaf(__uint_as_float(dpr[2 * t]), sc, -dvec_s[q0]);
+                    const float d1 = pv[q0 + 1] * fmaf(__uint_as_float(dpr[2 * t + 1]), sc, -dvec_s[q0 + 1]);
+                    w[t] = pack_bf16x2(d0, d1);
+                }
+                // packed over columns this group has already read
+                tmem_st16(tmem + lane_off + kColDP + c0 + h * 16, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        // ---- epilogue: dV, dK rows of this key block (summed over the group)
+        if (ok && n_it > 0) {
+            ok = mbar_wait(dkv_full, 0, abort_flag, kS1Compute);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const size_t row = static_cast<size_t>(bkv) * p.N + kv;
+                constexpr int kHalf = D / 2;
+#pragma unroll 1
+                for (int which = 0; which < 2; ++which) {
+                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kHalf;
+                    __nv_bfloat16* dst_row =
+                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kHalf;
+#pragma unroll 1
+                    for (int q = 0; q < kHalf / 32; ++q) {
+                        uint32_t v32[32];
+                        tmem_ld32(tmem + lane_off + col0 + q * 32, v32);
+                        tmem_ld_wait();
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t)
+                            pk[t] = pack_bf16x2(__uint_as_float(v32[2 * t]), __uint_as_float(v32[2 * t + 1]));
+                        if (kv_ok) {
+                            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
+#pragma unroll
+                            for (int t = 0; t < 4; ++t)
+                                dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ===========================================================================
+// dQ
+// ===========================================================================
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                 const BwdParams p) {
+    using L = DqLayout<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad + L::kBytes > static_cast<uint32_t>(L::kAlloc)) {
+        if (threadIdx.x == 0) atomicOr(&g_status, 1u << kS1Smem);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* q_full = bars + 0;     // Q and dO
+    uint64_t* k_full = bars + 1;     // [2]
+    uint64_t* v_full = bars + 3;     // [2]
+    uint64_t* kv_empty = bars + 5;   // [2]
+    uint64_t* s_full = bars + 7;
+    uint64_t* s_free = bars + 8;
+    uint64_t* dp_full = bars + 9;
+    uint64_t* ds_full = bars + 10;
+    uint64_t* dq_done = bars + 11;
+    uint64_t* drain = bars + 12;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // work unit: head groups; inside a group the heaviest (last) query tiles
+    // first, then the head
+    const int BH = p.B * p.Hq;
+    const int T = (p.N + kTileM - 1) / kTileM;
+    const int tile = static_cast<int>(blockIdx.x);
+    const int grp = tile / (p.dq_heads_per_group * T);
+    const int h0 = grp * p.dq_heads_per_group;
+    const int nh = min(p.dq_heads_per_group, BH - h0);
+    const int rr = tile - grp * p.dq_heads_per_group * T;
+    const int i = T - 1 - rr / nh;
+    const int bh = h0 + (rr % nh);
+    const int b = bh / p.Hq;
+    const int h = bh - b * p.Hq;
+    const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+    const int n_j = p.causal ? i + 1 : T;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, kCompute);
+        mbar_init(dp_full, 1);
+        mbar_init(ds_full, kCompute);
+        mbar_init(dq_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            tma_prefetch_desc(&tmDO);
+            mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+            for (int a = 0; a < D / 64; ++a) {
+                tma_load_3d(smem + L::kQ + a * L::kAtomBytes, &tmQ, q_full, a * 64, i * kTileM, bh);
+                tma_load_3d(smem + L::kDO + a * L::kAtomBytes, &tmDO, q_full, a * 64, i * kTileM, bh);
+            }
+            int issued = 0;
+            for (int jj = 0; jj < n_j; ++jj) {
+                const int st = jj & 1;
+                if (jj >= 2 && !mbar_wait(&kv_empty[st], ((jj >> 1) - 1) & 1, abort_flag, kS2Load)) break;
+                mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kK + st * L::kTileBytes + a * L::kAtomBytes, &tmK, &k_full[st], a * 64,
+                                jj * kTileN, kvh);
+                mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a)
+                    tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &v_full[st], a * 64,
+                                jj * kTileN, kvh);
+                issued = jj + 1;
+            }
+            wait_drain(q_full, 0, kS2Drain);
+            for (int jj = (issued > 2 ? issued - 2 : 0); jj < issued; ++jj) {
+                wait_drain(&k_full[jj & 1], (jj >> 1) & 1, kS2Drain);
+                wait_drain(&v_full[jj & 1], (jj >> 1) & 1, kS2Drain);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kTileN, 0, 0);  // S, dP: K-major both
+            constexpr uint32_t kIdDQ = idesc_bf16_f32(kTileM, D, 0, 1);     // dQ: A (dS) TMEM, B = K MN-major
+            const uint32_t q_base = smem_u32(smem + L::kQ);
+            const uint32_t do_base = smem_u32(smem + L::kDO);
+            const uint32_t k_base = smem_u32(smem + L::kK);
+            const uint32_t v_base = smem_u32(smem + L::kV);
+            constexpr uint32_t kAtom = L::kAtomBytes;
+            auto issue_s = [&](int st) {
+                const uint32_t ka = k_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    mma_ss(tmem + kColS, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), kIdS,
+                           kk > 0);
+                }
+                tc_commit(s_full);
+            };
+            auto issue_dp = [&](int st) {
+                const uint32_t va = v_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                    mma_ss(tmem + kColDP, sdesc_sw128(do_base + off, 16, 1024), sdesc_sw128(va + off, 16, 1024), kIdS,
+                           kk > 0);
+                }
+                tc_commit(dp_full);
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, kS2Load) && mbar_wait(&k_full[0], 0, abort_flag, kS2Load);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0);
+                ok = mbar_wait(&v_full[0], 0, abort_flag, kS2Load);
+                if (ok) {
+                    tc_fence_after();
+                    issue_dp(0);
+                }
+            }
+            for (int jj = 0; ok && jj < n_j; ++jj) {
+                const int st = jj & 1;
+                const uint32_t ph = jj & 1;
+                // S(j+1) once the compute warps have read S(j)
+                if (jj + 1 < n_j) {
+                    if (!(ok = mbar_wait(s_free, ph, abort_flag, kS2Mma))) break;
+                    if (!(ok = mbar_wait(&k_full[st ^ 1], ((jj + 1) >> 1) & 1, abort_flag, kS2Load))) break;
+                    tc_fence_after();
+                    issue_s(st ^ 1);
+                }
+                // dQ += dS K_j (dS packed as bf16 in the dP block)
+                if (!(ok = mbar_wait(ds_full, ph, abort_flag, kS2Mma))) break;
+                tc_fence_after();
+                const uint32_t ka = k_base + st * L::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 16; ++kk)
+                    mma_ts(tmem + kColDQ, tmem + kColDP + packed_col(kk), sdesc_sw128(ka + kk * 2048, kAtom, 1024),
+                           kIdDQ, (jj > 0 || kk > 0));
+                tc_commit(&kv_empty[st]);
+                // dP(j+1): its block held dS(j), consumed by the MMAs just issued
+                if (jj + 1 < n_j) {
+                    if (!(ok = mbar_wait(&v_full[st ^ 1], ((jj + 1) >> 1) & 1, abort_flag, kS2Load))) break;
+                    tc_fence_after();
+                    issue_dp(st ^ 1);
+                }
+            }
+            if (ok) tc_commit(dq_done);
+            tc_commit(drain);
+            wait_drain(drain, 0, kS2Drain);
+        }
+    } else {
+        // ------------------------------------------------------------ compute (P, dS)
+        const int wg = warp >> 2;
+        const int wq = warp & 3;
+        const int r = (wq << 5) + lane;  // query row of the tile = TMEM lane
+        const int qrow = i * kTileM + r;
+        const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
+        const int c0 = wg * 64;          // this group's key columns
+        const float c = p.scale_log2;
+        const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(qrow);
+        const float lse2 = p.lse2[srow];   // +inf on padding rows -> P = 0
+        const float dval = p.dvec[srow];   // scale * D
+        const float sc = p.scale;
+        float pv[64];
+        bool ok = true;
+        for (int jj = 0; jj < n_j; ++jj) {
+            const uint32_t ph = jj & 1;
+            ok = mbar_wait(s_full, ph, abort_flag, kS2Compute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            {
+                uint32_t sr[2][32];
+                tmem_ld32(tmem + lane_off + kColS + c0, sr[0]);
+                tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
+                tmem_ld_wait();
+                tc_fence_before();
+                mbar_arrive(s_free);
+                const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                const int kv0 = jj * kTileN + c0;
+                // Masked only on the causal diagonal tile and on a partial last
+                // key tile (uniform across the warp): key columns t >= hi are
+                // zero (past N, or after this query row on the diagonal).
+                const bool diag = p.causal && jj == i;
+                if (diag || kv0 + 64 > p.N) {
+                    const int hi = min(p.N, diag ? qrow + 1 : p.N) - kv0;
+                    static_for<0, 64>([&](auto tc) {
+                        constexpr int t = decltype(tc)::value;
+                        const float e = exp2_mixed<t>(fmaf(sv[t], c, -lse2));
+                        pv[t] = (t < hi) ? e : 0.f;
+                    });
+                } else {
+                    static_for<0, 64>([&](auto tc) {
+                        constexpr int t = decltype(tc)::value;
+                        pv[t] = exp2_mixed<t>(fmaf(sv[t], c, -lse2));
+                    });
+                }
+            }
+            ok = mbar_wait(dp_full, ph, abort_flag, kS2Compute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t dpr[32];
+                tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
+                tmem_ld_wait();
+                uint32_t w[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dval = scale*D
+                    const int q0 = hh * 32 + 2 * t;
+                    const float d0 = pv[q0] * fmaf(__uint_as_float(dpr[2 * t]), sc, -dval);
+                    const float d1 = pv[q0 + 1] * fmaf(__uint_as_float(dpr[2 * t + 1]), sc, -dval);
+                    w[t] = pack_bf16x2(d0, d1);
+                }
+                tmem_st16(tmem + lane_off + kColDP + c0 + hh * 16, w);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(ds_full);
+        }
+        // ---- epilogue: dQ rows (already scaled) -> bf16
+        if (ok && n_j > 0) {
+            ok = mbar_wait(dq_done, 0, abort_flag, kS2Compute);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                constexpr int kHalf = D / 2;
+                __nv_bfloat16* dst_row =
+                    reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(bh) * p.N + qrow) * D + wg * kHalf;
+#pragma unroll 1
+                for (int q = 0; q < kHalf / 32; ++q) {
+                    uint32_t v32[32];
+                    tmem_ld32(tmem + lane_off + kColDQ + wg * kHalf + q * 32, v32);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        pk[t] = pack_bf16x2(__uint_as_float(v32[2 * t]), __uint_as_float(v32[2 * t + 1]));
+                    if (qrow < p.N) {
+                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <class Kern>
+cudaError_t launch(Kern kern, unsigned grid, int smem, const CUtensorMap& tq, const CUtensorMap& tk,
+                   const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+    if (grid == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    kern<<<grid, kThreads, smem, stream>>>(tq, tk, tv, tdo, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+    const unsigned grid = static_cast<unsigned>((p.N + kTileN - 1) / kTileN) * p.B * p.Hkv;
+    if (D == 128) return launch(fa_bwd_dkdv_kernel<128>, grid, DkdvLayout<128>::kAlloc, tq, tk, tv, tdo, p, stream);
+    return launch(fa_bwd_dkdv_kernel<64>, grid, DkdvLayout<64>::kAlloc, tq, tk, tv, tdo, p, stream);
+}
+
+cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
+    const unsigned grid = static_cast<unsigned>((p.N + kTileM - 1) / kTileM) * p.B * p.Hq;
+    if (D == 128) return launch(fa_bwd_dq_kernel<128>, grid, DqLayout<128>::kAlloc, tq, tk, tv, tdo, p, stream);
+    return launch(fa_bwd_dq_kernel<64>, grid, DqLayout<64>::kAlloc, tq, tk, tv, tdo, p, stream);
+}
+
+}  // namespace fa

@@ -32,10 +32,12 @@ struct BwdParams {
     float scale;       // softmax scale (dS is pre-multiplied by it)
     float scale_log2;  // scale * log2(e)
     const float* lse2; // [B*Hq, Npad] lse * log2(e), +inf on padding rows
-    const float* dvec; // [B*Hq, Npad] D = rowsum(dO o O), 0 on padding rows
-    float* dq_acc;     // [B*Hq, N, D] fp32 accumulator
+    const float* dvec; // [B*Hq, Npad] scale * D, D = rowsum(dO o O); 0 on padding rows
+    float* dq_acc;     // [B*Hq, N, D] fp32 accumulator (fused kernel only)
+    void* dq;          // bf16 [B,Hq,N,D] (separate dQ pass writes it directly)
     void* dk;          // bf16 [B,Hkv,N,D]
     void* dv;          // bf16 [B,Hkv,N,D]
+    int dq_heads_per_group;  // query heads per scheduling group of the dQ pass
 };
 
 // Workspace carve-up for the backward (all offsets 256-byte aligned).
@@ -47,12 +49,20 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D);
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, cudaStream_t stream);
 
+// dq_acc == nullptr: do not zero a dQ accumulator (separate dQ pass).
 cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse,
                                   float* lse2, float* dvec, float* dq_acc,
-                                  int BH, int N, int Npad, cudaStream_t stream);
+                                  int BH, int N, int Npad, float scale, cudaStream_t stream);
 
+// Fused backward: dK, dV and dQ (fp32 reductions into p.dq_acc).
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
+
+// Separate-dQ backward: dK/dV kernel, then the dQ kernel writing p.dq.
+cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
+cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
 
 cudaError_t launch_bwd_dq_convert(const float* dq_acc, void* dq, size_t n_elems, cudaStream_t stream);
 

@@ -5,6 +5,7 @@
 #pragma once
 
 #include <cstdint>
+#include <type_traits>
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -239,6 +240,50 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA and integer pipes, leaving the MUFU unit to ex2() for the
+// other elements of a tile.  Cody-Waite style split x = n + f with
+// n = round(x) (added to 1.5*2^23 so the integer lands in the low mantissa
+// bits) and f in [-1/2, 1/2]; 2^f by a cubic whose coefficients were fitted
+// for minimum maximum relative error on [-1/2, 1/2] (see gen_exp2_poly.py:
+// 7.5e-5, below the 2^-9 rounding of the bf16 operands these values feed);
+// 2^n is applied by adding n to the exponent field.  Inputs below -125 are
+// clamped (result ~2^-125 instead of a smaller number or 0).
+__device__ __forceinline__ float exp2_fma(float x) {
+    x = fmaxf(x, -125.f);
+    const float t = x + 12582912.f;
+    const float n = t - 12582912.f;
+    const float f = x - n;
+    float p = fmaf(f, 0.0551716573536396f, 0.2426111400127411f);
+    p = fmaf(p, f, 0.6932609677314758f);
+    p = fmaf(p, f, 0.9999280571937561f);
+    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Share of a tile's exponentials computed by exp2_fma: elements whose index
+// modulo FA_EXP_POLY_DEN is below FA_EXP_POLY_NUM.
+#ifndef FA_EXP_POLY_NUM
+#define FA_EXP_POLY_NUM 0
+#endif
+#ifndef FA_EXP_POLY_DEN
+#define FA_EXP_POLY_DEN 2
+#endif
+// Compile-time unrolled loop: f(std::integral_constant<int, I>) for I in [B, E).
+template <int B, int E, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (B < E) {
+        f(std::integral_constant<int, B>{});
+        static_for<B + 1, E>(f);
+    }
+}
+
+template <int Q>
+__device__ __forceinline__ float exp2_mixed(float x) {
+    if constexpr ((Q % FA_EXP_POLY_DEN) < FA_EXP_POLY_NUM)
+        return exp2_fma(x);
+    else
+        return ex2(x);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
