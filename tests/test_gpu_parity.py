@@ -89,6 +89,30 @@ def test_small_shapes_full(B, Hq, Hkv, N, D, causal, scale, sqk):
         assert e <= G_TOL, f"{name} rel Frobenius err {e}"
 
 
+@pytest.mark.parametrize("mode", ["atomic", "separate"])
+def test_backward_dq_modes(mode):
+    """Both dQ strategies (fused kernel with fp32 reductions; separate dQ
+    pass) match the oracle and run the kernels they claim to."""
+    _gpu()
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, os.path.join(here, "_dq_mode_check.py")], env=dict(os.environ, FA_DQ_MODE=mode),
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+def test_backward_deterministic_separate_mode():
+    """The default backward has no reductions: repeated calls are bitwise equal."""
+    wl = WORKLOADS["tiny"].with_(causal=True, N=700, Hq=4, Hkv=2, D=128)
+    q, k, v, do = make_inputs(wl)
+    a = run(q, k, v, do, True, wl.softmax_scale)
+    b = run(q, k, v, do, True, wl.softmax_scale)
+    for t in ("dq", "dk", "dv"):
+        assert np.array_equal(a[t], b[t]), t
+
+
 def test_repeat_calls_identical_forward():
     wl = WORKLOADS["tiny"].with_(causal=True, N=333)
     q, k, v, do = make_inputs(wl)

@@ -270,49 +270,63 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tmem_ld_wait();
             float* sv = reinterpret_cast<float*>(&sr[0][0]);
             const int kv0 = j * kTileN;
-            const bool mask = (p.causal && j == nkv[s] - 1) || (kv0 + kTileN > p.N);
-            if (mask) {
+            // masked only on the causal diagonal tile and a partial last key
+            // tile (warp-uniform test): key columns >= hi get -inf
+            if ((p.causal && j == nkv[s] - 1) || (kv0 + kTileN > p.N)) {
+                const int hi = min(p.N, p.causal ? qrow + 1 : p.N) - kv0;
 #pragma unroll
-                for (int cix = 0; cix < 128; ++cix) {
-                    const int kv = kv0 + cix;
-                    if (kv >= p.N || (p.causal && kv > qrow)) sv[cix] = -INFINITY;
-                }
+                for (int cix = 0; cix < 128; ++cix) sv[cix] = (cix < hi) ? sv[cix] : -INFINITY;
             }
-            float mx = sv[0];
+            // row max with four independent chains
+            float mx4[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-            for (int cix = 1; cix < 128; ++cix) mx = fmaxf(mx, sv[cix]);
+            for (int cix = 4; cix < 128; cix += 4) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], sv[cix + u]);
+            }
+            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
             const float m_new = fmaxf(m_used, mx * c);
             const bool need = (m_new > m_used + kRescaleThreshold);
-            if (__any_sync(0xffffffffu, need)) {
-                const float alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
-                if (j > 0) {
-#pragma unroll 1
-                    for (int q = 0; q < D / 32; ++q) {
-                        uint32_t orow[32];
-                        tmem_ld32(tO + q * 32, orow);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int t = 0; t < 32; ++t)
-                            orow[t] = __float_as_uint(__uint_as_float(orow[t]) * alpha);
-                        tmem_st32(tO + q * 32, orow);
-                    }
-                }
+            // warp-uniform decision; alpha = 1 for rows whose max did not move
+            const bool rescale = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (rescale) {
+                alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
                 l *= alpha;
                 m_used = m_new;
             }
             const float msub = (m_used == -INFINITY) ? 0.f : m_used;
-            uint32_t pk[64];
-            float lsum = 0.f;
+            // P in two halves of 64 columns (packed into 32 TMEM columns each);
+            // the row sum uses four independent partial sums
+            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                const float p0 = ex2(fmaf(sv[2 * t], c, -msub));
-                const float p1 = ex2(fmaf(sv[2 * t + 1], c, -msub));
-                lsum += p0 + p1;
-                pk[t] = pack_bf16x2(p0, p1);
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int cix = half * 64 + 2 * t;
+                    const float p0 = ex2(fmaf(sv[cix], c, -msub));
+                    const float p1 = ex2(fmaf(sv[cix + 1], c, -msub));
+                    ls4[t & 3] += p0 + p1;
+                    pk[t] = pack_bf16x2(p0, p1);
+                }
+                tmem_st32(tS + half * 32, pk);
             }
-            l += lsum;
-            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+            l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+            // O <- alpha O (PV of the previous tile has completed: it was
+            // committed before this tile's S); done after P so the S row is
+            // no longer live in registers
+            if (rescale && j > 0) {
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t orow[32];
+                    tmem_ld32(tO + q * 32, orow);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) orow[t] = __float_as_uint(__uint_as_float(orow[t]) * alpha);
+                    tmem_st32(tO + q * 32, orow);
+                }
+            }
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_full[s]);
