@@ -96,26 +96,37 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- traffic record
+KERNEL_SOURCES = ("fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_split.cu", "sm100.cuh", "fa_internal.h")
+TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "dram_traffic_long.md")
+
+
 def kernel_source_hash() -> str:
+    """Hash of every source that decides what the kernels read and write
+    (the kernels and the launch configuration chosen by the API layer)."""
     h = hashlib.sha256()
-    for f in ("fa_bwd.cu", "fa_fwd.cu", "sm100.cuh", "fa_internal.h"):
+    for f in KERNEL_SOURCES:
         with open(os.path.join(ROOT, "tiled_attention_16_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
-    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
-    if not os.path.exists(path):
+    """DRAM bytes (read + write) per launch from the committed ncu summary,
+    or None when there is none for this kernel and workload or it was taken
+    on other kernel sources.  The summary's table rows read
+    `| kernel | workload | source hash | read bytes | write bytes | ... |`."""
+    if not os.path.exists(TRAFFIC_SUMMARY):
         return None
-    with open(path) as f:
-        d = json.load(f)
-    rec = d.get(kernel, {}).get(workload)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
-        return None
-    return rec.get("dram_bytes_per_launch")
+    src = kernel_source_hash()
+    with open(TRAFFIC_SUMMARY) as f:
+        for line in f:
+            cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 5 and cells[0] == kernel and cells[1] == workload and cells[2] == src:
+                try:
+                    return int(cells[3]) + int(cells[4])
+                except ValueError:
+                    return None
+    return None
 
 
 # ----------------------------------------------------------------------------- CPU oracle
