@@ -318,18 +318,18 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 // last key block (both uniform across the warp); there,
                 // columns q < lo are zero (lo = 64 masks a key row past N).
                 const bool diag = p.causal && (i == j);
+                const float2 c2 = make_float2(c, c);
+                static_for<0, 32>([&](auto tc) {
+                    constexpr int q = 2 * decltype(tc)::value;
+                    const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
+                    const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
+                    pv[q] = exp2_mixed<q>(x.x);
+                    pv[q + 1] = exp2_mixed<q + 1>(x.y);
+                });
                 if (diag || kv_block_partial) {
                     const int lo = !kv_ok ? 64 : (diag ? r - c0 : 0);
-                    static_for<0, 64>([&](auto qc) {
-                        constexpr int q = decltype(qc)::value;
-                        const float e = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
-                        pv[q] = (q >= lo) ? e : 0.f;
-                    });
-                } else {
-                    static_for<0, 64>([&](auto qc) {
-                        constexpr int q = decltype(qc)::value;
-                        pv[q] = exp2_mixed<q>(fmaf(sv[q], c, -lse_s[q]));
-                    });
+#pragma unroll
+                    for (int q = 0; q < 64; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
                 }
                 uint32_t pk[32];
 #pragma unroll
@@ -348,13 +348,16 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
                 tmem_ld_wait();
                 uint32_t w[16];
+                const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
                     const int q0 = h * 32 + 2 * t;
-                    const float d0 = pv[q0] * fmaf(__uint_as_float(dpr[2 * t]), sc, -dvec_s[q0]);
-                    const float d1 = pv[q0 + 1] * fmaf(__uint_as_float(dpr[2 * t + 1]), sc, -dvec_s[q0 + 1]);
-                    w[t] = pack_bf16x2(d0, d1);
+                    const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
+                    const float2 g = __ffma2_rn(make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])),
+                                                sc2, make_float2(-dv2.x, -dv2.y));
+                    const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), g);
+                    w[t] = pack_bf16x2(d.x, d.y);
                 }
                 // packed over columns this group has already read
                 tmem_st16(tmem + lane_off + kColDP + c0 + h * 16, w);
@@ -614,18 +617,18 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 // key tile (uniform across the warp): key columns t >= hi are
                 // zero (past N, or after this query row on the diagonal).
                 const bool diag = p.causal && jj == i;
+                const float2 c2 = make_float2(c, c);
+                const float2 nl2 = make_float2(-lse2, -lse2);
+                static_for<0, 32>([&](auto tc) {
+                    constexpr int t = 2 * decltype(tc)::value;
+                    const float2 x = __ffma2_rn(make_float2(sv[t], sv[t + 1]), c2, nl2);
+                    pv[t] = exp2_mixed<t>(x.x);
+                    pv[t + 1] = exp2_mixed<t + 1>(x.y);
+                });
                 if (diag || kv0 + 64 > p.N) {
                     const int hi = min(p.N, diag ? qrow + 1 : p.N) - kv0;
-                    static_for<0, 64>([&](auto tc) {
-                        constexpr int t = decltype(tc)::value;
-                        const float e = exp2_mixed<t>(fmaf(sv[t], c, -lse2));
-                        pv[t] = (t < hi) ? e : 0.f;
-                    });
-                } else {
-                    static_for<0, 64>([&](auto tc) {
-                        constexpr int t = decltype(tc)::value;
-                        pv[t] = exp2_mixed<t>(fmaf(sv[t], c, -lse2));
-                    });
+#pragma unroll
+                    for (int t = 0; t < 64; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
                 }
             }
             ok = mbar_wait(dp_full, ph, abort_flag, kS2Compute);
@@ -637,13 +640,16 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
                 tmem_ld_wait();
                 uint32_t w[16];
+                const float2 sc2 = make_float2(sc, sc);
+                const float2 nd2 = make_float2(-dval, -dval);
 #pragma unroll
                 for (int t = 0; t < 16; ++t) {
                     // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dval = scale*D
                     const int q0 = hh * 32 + 2 * t;
-                    const float d0 = pv[q0] * fmaf(__uint_as_float(dpr[2 * t]), sc, -dval);
-                    const float d1 = pv[q0 + 1] * fmaf(__uint_as_float(dpr[2 * t + 1]), sc, -dval);
-                    w[t] = pack_bf16x2(d0, d1);
+                    const float2 g = __ffma2_rn(make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])),
+                                                sc2, nd2);
+                    const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), g);
+                    w[t] = pack_bf16x2(d.x, d.y);
                 }
                 tmem_st16(tmem + lane_off + kColDP + c0 + hh * 16, w);
             }

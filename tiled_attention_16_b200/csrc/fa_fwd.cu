@@ -277,14 +277,16 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 #pragma unroll
                 for (int cix = 0; cix < 128; ++cix) sv[cix] = (cix < hi) ? sv[cix] : -INFINITY;
             }
-            // row max with four independent chains
+            // row max: four independent chains of three-input max
             float mx4[4] = {sv[0], sv[1], sv[2], sv[3]};
 #pragma unroll
-            for (int cix = 4; cix < 128; cix += 4) {
+            for (int cix = 4; cix < 124; cix += 8) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], sv[cix + u]);
+                for (int u = 0; u < 4; ++u) mx4[u] = fmax3(mx4[u], sv[cix + u], sv[cix + 4 + u]);
             }
-            const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], sv[124 + u]);
+            const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
             const float m_new = fmaxf(m_used, mx * c);
             const bool need = (m_new > m_used + kRescaleThreshold);
             // warp-uniform decision; alpha = 1 for rows whose max did not move
@@ -297,22 +299,25 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             }
             const float msub = (m_used == -INFINITY) ? 0.f : m_used;
             // P in two halves of 64 columns (packed into 32 TMEM columns each);
-            // the row sum uses four independent partial sums
-            float ls4[4] = {0.f, 0.f, 0.f, 0.f};
+            // scale-and-subtract and the row sum run on column pairs
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-msub, -msub);
+            float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t pk[32];
 #pragma unroll
                 for (int t = 0; t < 32; ++t) {
                     const int cix = half * 64 + 2 * t;
-                    const float p0 = ex2(fmaf(sv[cix], c, -msub));
-                    const float p1 = ex2(fmaf(sv[cix + 1], c, -msub));
-                    ls4[t & 3] += p0 + p1;
+                    const float2 x = __ffma2_rn(make_float2(sv[cix], sv[cix + 1]), c2, nm2);
+                    const float p0 = ex2(x.x);
+                    const float p1 = ex2(x.y);
+                    ls2[t & 1] = __fadd2_rn(ls2[t & 1], make_float2(p0, p1));
                     pk[t] = pack_bf16x2(p0, p1);
                 }
                 tmem_st32(tS + half * 32, pk);
             }
-            l += (ls4[0] + ls4[1]) + (ls4[2] + ls4[3]);
+            l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
             // O <- alpha O (PV of the previous tile has completed: it was
             // committed before this tile's S); done after P so the S row is
             // no longer live in registers
