@@ -323,6 +323,30 @@ def run_gpu(args, wl):
     }
     launches = sum(n for _, n in per_kernel.values())
 
+    # FP8 (e4m3) forward on the same workload, timed separately (not part of
+    # the step): tensor peak for e4m3 = measured bf16 peak x the nominal 2x ratio
+    if not args.no_fp8 and wl.D == 128:
+        from tiled_attention_16_b200.workloads import make_fp8_inputs
+        q8, k8, v8, qs, ks, vs = make_fp8_inputs(rank_workload(wl, rank))
+        q8, k8, v8 = q8.to(dev), k8.to(dev), v8.to(dev)
+        o8 = torch.empty_like(o)
+        for _ in range(3):
+            A.fwd_fp8(q8, k8, v8, qs, ks, vs, causal=wl.causal, out=o8, lse=lse)
+        torch.cuda.synchronize()
+        A.profile_begin()
+        for _ in range(20):
+            A.fwd_fp8(q8, k8, v8, qs, ks, vs, causal=wl.causal, out=o8, lse=lse)
+        t8, n8 = A.profile_end()["fa_fwd_fp8_kernel"]
+        if A.device_status(dev) != A.FA_OK:
+            raise RuntimeError("device status not OK after the FP8 forward")
+        f8_ms = t8 / n8
+        f8_tf = wl.flops_fwd() / (f8_ms * 1e-3) / 1e12
+        breakdown["fp8_fwd"] = {"ms": f8_ms, "tflops": f8_tf, "peak": 2 * peak_tf,
+                                "frac_of_peak": f8_tf / (2 * peak_tf),
+                                "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3/bf16 ratio)",
+                                "launches": n8, "timed_alone": True}
+        del q8, k8, v8, o8
+
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -394,6 +418,7 @@ def main():
     ap.add_argument("--workload", default="long")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the separate FP8 forward measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

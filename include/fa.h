@@ -75,6 +75,20 @@ typedef struct {
 FA_API fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void* v,
                  void* o, float* lse, void* stream);
 
+/* FP8 forward (FlashAttention-3's FP8 operands, named in "【词汇专栏】
+ * FlashAttention：大模型训练的加速器", section 3.3; the scaling convention is
+ * this library's).  q [B,Hq,N,D], k/v [B,Hkv,N,D] hold e4m3 bytes (OCP FP8
+ * E4M3, finite-only, 1 byte per element, contiguous); the value each element
+ * stands for is element * q_scale (k_scale, v_scale), all three finite and
+ * > 0.  Computes the same O and LSE as fa_fwd over those values: o
+ * [B,Hq,N,D] bf16 and lse [B,Hq,N] fp32.  Both products run on the 8-bit
+ * tensor-core path with fp32 accumulation; the probabilities are rounded to
+ * e4m3 for the P V product (the row sums use them unrounded), so O carries a
+ * relative error of up to 2^-4 per probability term.  D = 128 only
+ * (FA_ERR_UNSUPPORTED otherwise).  Asynchronous on `stream` like fa_fwd. */
+FA_API fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const void* v,
+                     float q_scale, float k_scale, float v_scale, void* o, float* lse, void* stream);
+
 /* Bytes of device workspace fa_bwd needs for `shape` (0 if the shape is invalid):
  * the per-row statistics (LSE in log2 units and D = rowsum(dO o O), each
  * padded to a multiple of 128 rows) and an fp32 dQ accumulator [B,Hq,N,D]. */
@@ -135,11 +149,11 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * kernel kind k the summed duration total_ms[k] and the launch count
  * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
  * preprocess, 2 fused backward (dK, dV and dQ by fp32 reductions), 3 dQ
- * convert, 4 backward dK/dV kernel, 5 backward dQ kernel (FA_PROFILE_KINDS;
+ * convert, 4 backward dK/dV kernel, 5 backward dQ kernel, 6 FP8 forward (FA_PROFILE_KINDS;
  * fa_bwd uses 1, 4, 5 by default and 1, 2, 3 when the environment variable
  * FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
  * objects; no device memory is allocated. */
-#define FA_PROFILE_KINDS 6
+#define FA_PROFILE_KINDS 7
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

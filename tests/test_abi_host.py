@@ -19,7 +19,7 @@ def test_exports_every_declared_symbol():
     names = A.declared_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
                           "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
-                          "fa_bwd_noalloc"}
+                          "fa_bwd_noalloc", "fa_fwd_fp8"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -36,6 +36,10 @@ P = 0x10000  # fake, 16-byte-aligned "device" address; never dereferenced on rej
 
 def _fwd(shape, q=P, k=P, v=P, o=P, lse=P):
     return A.lib().fa_fwd(None if shape is None else ctypes.byref(shape), q, k, v, o, lse, None)
+
+
+def _fwd8(shape, q=P, k=P, v=P, o=P, lse=P, qs=1.0, ks=1.0, vs=1.0):
+    return A.lib().fa_fwd_fp8(None if shape is None else ctypes.byref(shape), q, k, v, qs, ks, vs, o, lse, None)
 
 
 def _bwd(shape, ws=P, ws_bytes=1 << 40, ptr=P, **over):
@@ -123,7 +127,7 @@ def test_profile_hooks_without_launches():
     A.profile_begin()
     res = A.profile_end()
     assert set(res) == set(A.PROFILE_KINDS)
-    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 6
+    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 7
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
 
 
@@ -142,3 +146,24 @@ def test_noalloc_host_checks():
     big = A.make_shape(1, 32, 32, 4096, 128, 0.1, 1)
     assert A.lib().fa_bwd_workspace_bytes(ctypes.byref(big)) > A.NOALLOC_SCRATCH_BYTES
     assert _noalloc(big) == A.FA_ERR_TOO_LARGE
+
+
+def test_fp8_forward_host_checks():
+    assert _fwd8(None) == A.FA_ERR_INVALID_ARG
+    assert _fwd8(shape(N=0)) == A.FA_ERR_INVALID_ARG
+    assert _fwd8(shape(Hq=3, Hkv=2)) == A.FA_ERR_INVALID_ARG
+    assert _fwd8(shape(D=64)) == A.FA_ERR_UNSUPPORTED      # e4m3 path: D = 128 only
+    assert _fwd8(shape(D=96)) == A.FA_ERR_UNSUPPORTED
+    for bad in (0.0, -1.0, float("nan"), float("inf")):
+        for which in ("qs", "ks", "vs"):
+            assert _fwd8(shape(), **{which: bad}) == A.FA_ERR_INVALID_ARG
+    for which in ("q", "k", "v", "o", "lse"):
+        assert _fwd8(shape(), **{which: P + 8}) == A.FA_ERR_INVALID_ARG
+        assert _fwd8(shape(), **{which: 0}) == A.FA_ERR_INVALID_ARG
+
+
+def test_fp8_binding_checks_dtype():
+    import torch
+    q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        A.fwd_fp8(q, q, q)

@@ -48,6 +48,9 @@ def lib() -> ctypes.CDLL:
         vp, sz = ctypes.c_void_p, ctypes.c_size_t
         shp = ctypes.POINTER(FaShape)
         L.fa_fwd.argtypes = [shp, vp, vp, vp, vp, vp, vp]
+        f32 = ctypes.c_float
+        L.fa_fwd_fp8.argtypes = [shp, vp, vp, vp, f32, f32, f32, vp, vp, vp]
+        L.fa_fwd_fp8.restype = ctypes.c_int
         L.fa_fwd.restype = ctypes.c_int
         L.fa_bwd_workspace_bytes.argtypes = [shp]
         L.fa_bwd_workspace_bytes.restype = sz
@@ -131,6 +134,31 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     return out, lse
 
 
+def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_scale: float = 1.0, k_scale: float = 1.0,
+            v_scale: float = 1.0, causal: bool = False, scale: float | None = None,
+            out: torch.Tensor | None = None, lse: torch.Tensor | None = None):
+    """FP8 attention forward over e4m3 tensors (torch.float8_e4m3fn), each
+    element standing for element * its tensor's descale.  Returns (o bf16,
+    lse fp32) as fwd() does.  Head dimension 128 only."""
+    B, Hq, Hkv, N, D = _dims(q8, k8)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(q8, "q8", (B, Hq, N, D), torch.float8_e4m3fn)
+    _check(k8, "k8", (B, Hkv, N, D), torch.float8_e4m3fn)
+    _check(v8, "v8", (B, Hkv, N, D), torch.float8_e4m3fn)
+    if out is None:
+        out = torch.empty((B, Hq, N, D), device=q8.device, dtype=torch.bfloat16)
+    if lse is None:
+        lse = torch.empty((B, Hq, N), device=q8.device, dtype=torch.float32)
+    _check(out, "out", (B, Hq, N, D))
+    _check(lse, "lse", (B, Hq, N), torch.float32)
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    st = lib().fa_fwd_fp8(ctypes.byref(shp), q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(q_scale),
+                          float(k_scale), float(v_scale), out.data_ptr(), lse.data_ptr(), _stream_ptr(q8.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_fp8")
+    return out, lse
+
+
 def workspace_bytes(B, Hq, Hkv, N, D, causal=False, scale=None) -> int:
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
@@ -203,7 +231,7 @@ def timeout_sites() -> int:
 
 
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
-                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel")
+                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel")
 
 
 def profile_begin() -> None:

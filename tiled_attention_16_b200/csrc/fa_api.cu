@@ -33,16 +33,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// 3-D map over a contiguous bf16 [BH, N, D] tensor: box = 64 columns x 128
-// rows x 1 head, 128-byte swizzle; rows past N read as zero.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D) {
+// 3-D map over a contiguous [BH, N, D] tensor: box = 128 bytes of a row
+// (64 bf16 or 128 e4m3) x 128 rows x 1 head, 128-byte swizzle; rows past N
+// read as zero.
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int elem_bytes = 2) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(N) * D * 2};
-    cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kTileM), 1};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * eb, static_cast<cuuint64_t>(N) * D * eb};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(kTileM), 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+    const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
@@ -212,8 +215,45 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     }
     p.o = o;
     p.lse = lse;
+    p.o_scale = 1.f;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const void* v, float q_scale,
+                     float k_scale, float v_scale, void* o, float* lse, void* stream) {
+    fa_status st = check_shape(shape);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+    for (float x : {q_scale, k_scale, v_scale})
+        if (!std::isfinite(x) || !(x > 0.f)) return FA_ERR_INVALID_ARG;
+    if (shape->D != 128) return FA_ERR_UNSUPPORTED;
+    if ((st = check_device()) != FA_OK) return st;
+    const fa_shape& s = *shape;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D, 1) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D, 1) ||
+        !make_map(&tv, v, s.B * s.Hkv, s.N, s.D, 1))
+        return FA_ERR_CUDA;
+    FwdParams p;
+    p.B = s.B;
+    p.Hq = s.Hq;
+    p.Hkv = s.Hkv;
+    p.N = s.N;
+    p.causal = s.causal ? 1 : 0;
+    p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634 * q_scale * k_scale);
+    p.n_mblocks = (s.N + 2 * kTileM - 1) / (2 * kTileM);
+    {
+        // e4m3 K/V: half the bytes of bf16 per head, same ~32 MiB L2 budget
+        const double per_head = 2.0 * s.N * s.D / (s.Hq / s.Hkv);
+        const int g = static_cast<int>(32.0 * 1024 * 1024 / per_head);
+        p.heads_per_group = g < 1 ? 1 : (g > s.B * s.Hq ? s.B * s.Hq : g);
+    }
+    p.o = o;
+    p.lse = lse;
+    p.o_scale = v_scale;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed(6, strm, [&] { return launch_fwd_fp8(tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -35,8 +35,16 @@ namespace fa {
 
 namespace {
 
-constexpr int kThreads = 320;
-constexpr int kCompute = 256;
+// Compute warps form kGroups groups of four (one warp per TMEM lane quarter);
+// group g owns kCols consecutive columns of the 128-column score tile.
+constexpr int kGroups = 2;
+constexpr int kCols = kTileN / kGroups;
+constexpr int kComputeWarps = 4 * kGroups;
+constexpr int kMmaWarp = kComputeWarps;
+constexpr int kLoadWarp = kComputeWarps + 1;
+constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kCompute = 32 * kComputeWarps;
+static_assert(kCols % 32 == 0, "each compute thread handles whole 32-column TMEM loads");
 constexpr int kMaxDynSmem = 232448;
 
 // wait sites (bits of the device status word)
@@ -46,9 +54,12 @@ enum SplitSite {
 };
 
 // TMEM column (relative to a 128-column block) of K-step kk (16 columns of
-// the score tile) of a bf16 operand packed by the two compute groups: group g
-// packs its 64 columns into block columns [64g, 64g + 32).
-__host__ __device__ constexpr uint32_t packed_col(int kk) { return (kk >> 2) * 64 + (kk & 3) * 8; }
+// the score tile) of a bf16 operand packed by the compute groups: group g
+// packs its kCols columns into block columns [g kCols, g kCols + kCols / 2),
+// columns it has itself already read.
+__host__ __device__ constexpr uint32_t packed_col(int kk) {
+    return static_cast<uint32_t>((kk / (kCols / 16)) * kCols + (kk % (kCols / 16)) * 8);
+}
 
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int site) {
     if (mbar_try_wait(bar, parity)) return;
@@ -175,7 +186,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
-    if (warp == 9) {
+    if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -215,7 +226,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (int it = (issued_do > 2 ? issued_do - 2 : 0); it < issued_do; ++it)
                 wait_drain(&do_full[it & 1], (it >> 1) & 1, kS1Drain);
         }
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdSq = idesc_bf16_f32(kTileN, kTileM, 0, 0);  // S^T, dP^T
@@ -290,12 +301,12 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int r = (wq << 5) + lane;  // key row of the block = TMEM lane
         const int kv = j * kTileN + r;
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
-        const int c0 = wg * 64;          // this group's query columns
+        const int c0 = wg * kCols;       // this group's query columns
         const float c = p.scale_log2;
         const float sc = p.scale;
         const bool kv_ok = kv < p.N;
         const bool kv_block_partial = (j + 1) * kTileN > p.N;
-        float pv[64];
+        float pv[kCols];
         bool ok = true;
         for (int it = 0; it < n_it; ++it) {
             const int st = it & 1;
@@ -309,17 +320,17 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             {
-                uint32_t sr[2][32];
-                tmem_ld32(tmem + lane_off + kColS + c0, sr[0]);
-                tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
+                uint32_t sr[kCols / 32][32];
+#pragma unroll
+                for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
                 tmem_ld_wait();
                 const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
                 // Masked only on the causal diagonal block and on a partial
                 // last key block (both uniform across the warp); there,
-                // columns q < lo are zero (lo = 64 masks a key row past N).
+                // columns q < lo are zero (lo = kCols masks a key row past N).
                 const bool diag = p.causal && (i == j);
                 const float2 c2 = make_float2(c, c);
-                static_for<0, 32>([&](auto tc) {
+                static_for<0, kCols / 2>([&](auto tc) {
                     constexpr int q = 2 * decltype(tc)::value;
                     const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
                     const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
@@ -327,14 +338,17 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     pv[q + 1] = exp2_mixed<q + 1>(x.y);
                 });
                 if (diag || kv_block_partial) {
-                    const int lo = !kv_ok ? 64 : (diag ? r - c0 : 0);
+                    const int lo = !kv_ok ? kCols : (diag ? r - c0 : 0);
 #pragma unroll
-                    for (int q = 0; q < 64; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
+                    for (int q = 0; q < kCols; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
                 }
-                uint32_t pk[32];
 #pragma unroll
-                for (int t = 0; t < 32; ++t) pk[t] = pack_bf16x2(pv[2 * t], pv[2 * t + 1]);
-                tmem_st32(tmem + lane_off + kColS + c0, pk);
+                for (int h = 0; h < kCols / 32; ++h) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pv[32 * h + 2 * t], pv[32 * h + 2 * t + 1]);
+                    tmem_st16(tmem + lane_off + kColS + c0 + h * 16, pk);
+                }
                 tmem_st_wait();
             }
             tc_fence_before();
@@ -343,7 +357,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            for (int h = 0; h < kCols / 32; ++h) {
                 uint32_t dpr[32];
                 tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
                 tmem_ld_wait();
@@ -372,26 +386,25 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
                 const size_t row = static_cast<size_t>(bkv) * p.N + kv;
-                constexpr int kHalf = D / 2;
+                constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
 #pragma unroll 1
                 for (int which = 0; which < 2; ++which) {
-                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kHalf;
+                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
                     __nv_bfloat16* dst_row =
-                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kHalf;
+                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kPer;
 #pragma unroll 1
-                    for (int q = 0; q < kHalf / 32; ++q) {
-                        uint32_t v32[32];
-                        tmem_ld32(tmem + lane_off + col0 + q * 32, v32);
+                    for (int q = 0; q < kPer / 16; ++q) {
+                        uint32_t v16[16];
+                        tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
                         tmem_ld_wait();
-                        uint32_t pk[16];
+                        uint32_t pk[8];
 #pragma unroll
-                        for (int t = 0; t < 16; ++t)
-                            pk[t] = pack_bf16x2(__uint_as_float(v32[2 * t]), __uint_as_float(v32[2 * t + 1]));
+                        for (int t = 0; t < 8; ++t)
+                            pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
                         if (kv_ok) {
-                            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
-#pragma unroll
-                            for (int t = 0; t < 4; ++t)
-                                dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                         }
                     }
                 }
@@ -482,7 +495,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
 
-    if (warp == 9) {
+    if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
@@ -514,7 +527,7 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 wait_drain(&v_full[jj & 1], (jj >> 1) & 1, kS2Drain);
             }
         }
-    } else if (warp == 8) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t kIdS = idesc_bf16_f32(kTileM, kTileN, 0, 0);  // S, dP: K-major both
@@ -591,13 +604,13 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int r = (wq << 5) + lane;  // query row of the tile = TMEM lane
         const int qrow = i * kTileM + r;
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
-        const int c0 = wg * 64;          // this group's key columns
+        const int c0 = wg * kCols;       // this group's key columns
         const float c = p.scale_log2;
         const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(qrow);
         const float lse2 = p.lse2[srow];   // +inf on padding rows -> P = 0
         const float dval = p.dvec[srow];   // scale * D
         const float sc = p.scale;
-        float pv[64];
+        float pv[kCols];
         bool ok = true;
         for (int jj = 0; jj < n_j; ++jj) {
             const uint32_t ph = jj & 1;
@@ -605,9 +618,9 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
             {
-                uint32_t sr[2][32];
-                tmem_ld32(tmem + lane_off + kColS + c0, sr[0]);
-                tmem_ld32(tmem + lane_off + kColS + c0 + 32, sr[1]);
+                uint32_t sr[kCols / 32][32];
+#pragma unroll
+                for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
                 tmem_ld_wait();
                 tc_fence_before();
                 mbar_arrive(s_free);
@@ -619,23 +632,23 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 const bool diag = p.causal && jj == i;
                 const float2 c2 = make_float2(c, c);
                 const float2 nl2 = make_float2(-lse2, -lse2);
-                static_for<0, 32>([&](auto tc) {
+                static_for<0, kCols / 2>([&](auto tc) {
                     constexpr int t = 2 * decltype(tc)::value;
                     const float2 x = __ffma2_rn(make_float2(sv[t], sv[t + 1]), c2, nl2);
                     pv[t] = exp2_mixed<t>(x.x);
                     pv[t + 1] = exp2_mixed<t + 1>(x.y);
                 });
-                if (diag || kv0 + 64 > p.N) {
+                if (diag || kv0 + kCols > p.N) {
                     const int hi = min(p.N, diag ? qrow + 1 : p.N) - kv0;
 #pragma unroll
-                    for (int t = 0; t < 64; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
+                    for (int t = 0; t < kCols; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
                 }
             }
             ok = mbar_wait(dp_full, ph, abort_flag, kS2Compute);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
+            for (int hh = 0; hh < kCols / 32; ++hh) {
                 uint32_t dpr[32];
                 tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
                 tmem_ld_wait();
@@ -662,23 +675,22 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             ok = mbar_wait(dq_done, 0, abort_flag, kS2Compute);
             if (__all_sync(0xffffffffu, ok)) {
                 tc_fence_after();
-                constexpr int kHalf = D / 2;
+                constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
                 __nv_bfloat16* dst_row =
-                    reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(bh) * p.N + qrow) * D + wg * kHalf;
+                    reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(bh) * p.N + qrow) * D + wg * kPer;
 #pragma unroll 1
-                for (int q = 0; q < kHalf / 32; ++q) {
-                    uint32_t v32[32];
-                    tmem_ld32(tmem + lane_off + kColDQ + wg * kHalf + q * 32, v32);
+                for (int q = 0; q < kPer / 16; ++q) {
+                    uint32_t v16[16];
+                    tmem_ld16(tmem + lane_off + kColDQ + wg * kPer + q * 16, v16);
                     tmem_ld_wait();
-                    uint32_t pk[16];
+                    uint32_t pk[8];
 #pragma unroll
-                    for (int t = 0; t < 16; ++t)
-                        pk[t] = pack_bf16x2(__uint_as_float(v32[2 * t]), __uint_as_float(v32[2 * t + 1]));
+                    for (int t = 0; t < 8; ++t)
+                        pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
                     if (qrow < p.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 32);
-#pragma unroll
-                        for (int t = 0; t < 4; ++t)
-                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
                 }
             }

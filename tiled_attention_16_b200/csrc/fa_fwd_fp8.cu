@@ -1,0 +1,404 @@
+// fa_fwd_fp8.cu — tiled attention forward with FP8 (e4m3) Q, K, V for sm_100a.
+//
+// The same tiling and incremental softmax as fa_fwd.cu ("【词汇专栏】
+// FlashAttention：大模型训练的加速器", sections 2.1-2.3; FP8 operands are the
+// FlashAttention-3 feature its section 3.3 names), with both products on the
+// 8-bit tensor-core path (tcgen05.mma kind::f8f6f4, fp32 accumulation):
+//
+//   S = Q K^T            e4m3 x e4m3 -> fp32; the per-tensor descales of Q and
+//                        K are folded into the softmax constant
+//   P = 2^(S c - m)      fp32, row sum l taken from these fp32 values
+//   O += P8 V            P rounded to e4m3 (RNE, saturating) and read from
+//                        tensor memory as the A operand; V e4m3 from shared memory
+//   O = O * v_scale / l  bf16 output, LSE in fp32 (natural log) as for bf16
+//
+// Layout: an e4m3 tile of 128 rows x 128 columns is exactly one 128-byte
+// swizzle atom column (16 KB), so a K step of 32 elements advances 32 bytes
+// (Q, K: K-major) or 32 rows = 4 KB (V: MN-major).  P is packed four keys per
+// 32-bit tensor-memory column (key 4w + b in byte b of column w), over the
+// first 32 columns of its own S block.
+//
+// Warp roles (320 threads) as in the bf16 kernel: warps 0-3 / 4-7 softmax for
+// query tiles 0 / 1, warp 8 MMA issuer, warp 9 TMA producer (Q once, K/V
+// through a three-stage ring).  Head dimension 128 only.
+#include "fa_internal.h"
+#include "sm100.cuh"
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+namespace fa {
+
+namespace {
+
+constexpr int kF8Threads = 320;
+constexpr int kF8Stages = 3;
+constexpr int kF8D = 128;
+constexpr float kF8RescaleThreshold = 8.0f;
+
+// wait sites: the bits of the bf16 forward (a timeout names the same stage)
+enum F8Site { kF8Q = 0, kF8K = 1, kF8V = 2, kF8KVEmpty = 3, kF8S = 4, kF8P = 5, kF8O = 6, kF8Drain = 7 };
+
+struct F8Layout {
+    static constexpr int kTileBytes = kTileM * kF8D;  // 128 rows x 128 e4m3
+    static constexpr int kQ = 0;                       // 2 tiles
+    static constexpr int kK = kQ + 2 * kTileBytes;     // kF8Stages tiles
+    static constexpr int kV = kK + kF8Stages * kTileBytes;
+    static constexpr int kBar = kV + kF8Stages * kTileBytes;
+    static constexpr int kNumBars = 1 + 3 * kF8Stages + 3 * 2 + 1;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A and B (format code 0) and
+// fp32 accumulation; a_mn / b_mn select MN-major operands.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N, int a_mn, int b_mn) {
+    return (1u << 4)
+         | (static_cast<uint32_t>(a_mn) << 15)
+         | (static_cast<uint32_t>(b_mn) << 16)
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Four probabilities -> one word of e4m3 bytes, the first in the low byte.
+__device__ __forceinline__ uint32_t pack_e4m3x4(float p0, float p1, float p2, float p3) {
+    const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(p0, p1), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(p2, p3), __NV_SATFINITE, __NV_E4M3);
+    return lo | (hi << 16);
+}
+
+__device__ __forceinline__ float lg2f(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void f8_wait_drain(uint64_t* bar, uint32_t parity, int site) {
+    if (mbar_try_wait(bar, parity)) return;
+    unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return;
+        if ((it & 63u) == 0 && globaltimer_ns() - t0 > kWaitLimitNs) {
+            atomicOr(&g_status, 1u << site);
+            return;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kF8Threads, 1)
+fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+    using L = F8Layout;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* q_full = bars + 0;
+    uint64_t* k_full = bars + 1;                    // [kF8Stages]
+    uint64_t* v_full = k_full + kF8Stages;          // [kF8Stages]
+    uint64_t* kv_empty = v_full + kF8Stages;        // [kF8Stages]
+    uint64_t* s_full = kv_empty + kF8Stages;        // [2]
+    uint64_t* p_full = s_full + 2;                  // [2]
+    uint64_t* o_full = p_full + 2;                  // [2]
+    uint64_t* drain = o_full + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // work unit: head groups, heaviest causal query block first (as in bf16)
+    const int BH = p.B * p.Hq;
+    const int tile = static_cast<int>(blockIdx.x);
+    const int grp = tile / (p.heads_per_group * p.n_mblocks);
+    const int h_first = grp * p.heads_per_group;
+    const int nh = min(p.heads_per_group, BH - h_first);
+    const int rr = tile - grp * p.heads_per_group * p.n_mblocks;
+    const int mb = p.n_mblocks - 1 - rr / nh;
+    const int bh = h_first + rr % nh;
+    const int b = bh / p.Hq;
+    const int h = bh - b * p.Hq;
+    const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+    const int m0 = mb * 2 * kTileM;
+    const int n_kv_total = (p.N + kTileN - 1) / kTileN;
+    const bool act1 = (m0 + kTileM) < p.N;
+    int nkv[2];
+    if (p.causal) {
+        nkv[0] = 2 * mb + 1;
+        nkv[1] = act1 ? 2 * mb + 2 : 0;
+    } else {
+        nkv[0] = n_kv_total;
+        nkv[1] = act1 ? n_kv_total : 0;
+    }
+    const int n_iter = act1 ? nkv[1] : nkv[0];
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < kF8Stages; ++s) {
+            mbar_init(&k_full[s], 1);
+            mbar_init(&v_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], kTileM);
+            mbar_init(&o_full[s], 1);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 9) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            const int nsub = act1 ? 2 : 1;
+            mbar_arrive_expect_tx(q_full, nsub * L::kTileBytes);
+            for (int s = 0; s < nsub; ++s)
+                tma_load_3d(smem + L::kQ + s * L::kTileBytes, &tmQ, q_full, 0, m0 + s * kTileM, bh);
+            int issued = 0;
+            for (int j = 0; j < n_iter; ++j) {
+                const int st = j % kF8Stages;
+                if (j >= kF8Stages &&
+                    !mbar_wait(&kv_empty[st], ((j / kF8Stages) - 1) & 1, abort_flag, kF8KVEmpty))
+                    break;
+                mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                tma_load_3d(smem + L::kK + st * L::kTileBytes, &tmK, &k_full[st], 0, j * kTileN, kvh);
+                mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
+                tma_load_3d(smem + L::kV + st * L::kTileBytes, &tmV, &v_full[st], 0, j * kTileN, kvh);
+                issued = j + 1;
+            }
+            f8_wait_drain(q_full, 0, kF8Drain);
+            for (int j = (issued > kF8Stages ? issued - kF8Stages : 0); j < issued; ++j) {
+                f8_wait_drain(&k_full[j % kF8Stages], (j / kF8Stages) & 1, kF8Drain);
+                f8_wait_drain(&v_full[j % kF8Stages], (j / kF8Stages) & 1, kF8Drain);
+            }
+        }
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t kIdS = idesc_e4m3_f32(kTileM, kTileN, 0, 0);
+            constexpr uint32_t kIdPV = idesc_e4m3_f32(kTileM, kF8D, 0, 1);
+            const uint64_t q_desc = sdesc_sw128(smem_u32(smem + L::kQ), 16, 1024);            // K-major
+            const uint64_t k_desc = sdesc_sw128(smem_u32(smem + L::kK), 16, 1024);            // K-major
+            const uint64_t v_desc = sdesc_sw128(smem_u32(smem + L::kV), L::kTileBytes, 1024);  // MN-major
+            auto issue_s = [&](int s, int st) {
+                const uint64_t qd = q_desc + ((s * L::kTileBytes) >> 4);
+                const uint64_t kd = k_desc + ((st * L::kTileBytes) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < kF8D / 32; ++kk)  // 32 e4m3 = 32 bytes per K step
+                    mma_f8_ss(tmem + s * 128, qd + ((kk * 32) >> 4), kd + ((kk * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
+            };
+            auto issue_pv = [&](int s, int st, int j) {
+                const uint64_t vd = v_desc + ((st * L::kTileBytes) >> 4);
+                const uint32_t acc0 = j > 0 ? 1u : 0u;
+#pragma unroll
+                for (int kk = 0; kk < kTileN / 32; ++kk)  // 32 keys = 8 packed columns = 32 V rows
+                    mma_f8_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, vd + ((kk * 32 * 128) >> 4), kIdPV,
+                              kk > 0 ? 1u : acc0);
+            };
+            bool ok = mbar_wait(q_full, 0, abort_flag, kF8Q) && mbar_wait(&k_full[0], 0, abort_flag, kF8K);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                tc_commit(&s_full[0]);
+                if (nkv[1] > 0) {
+                    issue_s(1, 0);
+                    tc_commit(&s_full[1]);
+                }
+            }
+            for (int j = 0; ok && j < n_iter; ++j) {
+                const int st = j % kF8Stages;
+                const int sn = (j + 1) % kF8Stages;
+                const uint32_t sn_ph = ((j + 1) / kF8Stages) & 1;
+                if (!(ok = mbar_wait(&v_full[st], (j / kF8Stages) & 1, abort_flag, kF8V))) break;
+                if (j < nkv[0]) {
+                    if (!(ok = mbar_wait(&p_full[0], j & 1, abort_flag, kF8P))) break;
+                    tc_fence_after();
+                    issue_pv(0, st, j);
+                    if (j == nkv[0] - 1) tc_commit(&o_full[0]);
+                    if (j + 1 < nkv[0]) {
+                        if (!(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
+                        tc_fence_after();
+                        issue_s(0, sn);
+                        tc_commit(&s_full[0]);
+                    }
+                }
+                if (j < nkv[1]) {
+                    if (!(ok = mbar_wait(&p_full[1], j & 1, abort_flag, kF8P))) break;
+                    tc_fence_after();
+                    issue_pv(1, st, j);
+                    if (j == nkv[1] - 1) tc_commit(&o_full[1]);
+                }
+                tc_commit(&kv_empty[st]);
+                if (j + 1 < nkv[1]) {
+                    if (!(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
+                    tc_fence_after();
+                    issue_s(1, sn);
+                    tc_commit(&s_full[1]);
+                }
+            }
+            tc_commit(drain);
+            f8_wait_drain(drain, 0, kF8Drain);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const int s = warp >> 2;
+        const int r = ((warp & 3) << 5) + lane;
+        const int qrow = m0 + s * kTileM + r;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) << 5) << 16;
+        const uint32_t tS = tmem + lane_off + s * 128;
+        const uint32_t tO = tmem + lane_off + 256 + s * 128;
+        const float c = p.scale_log2;  // scale * log2(e) * q_scale * k_scale
+        float m_used = -INFINITY;
+        float l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv[s]; ++j) {
+            ok = mbar_wait(&s_full[s], j & 1, abort_flag, kF8S);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+            tmem_ld_wait();
+            float* sv = reinterpret_cast<float*>(&sr[0][0]);
+            const int kv0 = j * kTileN;
+            if ((p.causal && j == nkv[s] - 1) || (kv0 + kTileN > p.N)) {
+                const int hi = min(p.N, p.causal ? qrow + 1 : p.N) - kv0;
+#pragma unroll
+                for (int cix = 0; cix < 128; ++cix) sv[cix] = (cix < hi) ? sv[cix] : -INFINITY;
+            }
+            float mx4[4] = {sv[0], sv[1], sv[2], sv[3]};
+#pragma unroll
+            for (int cix = 4; cix < 124; cix += 8) {
+#pragma unroll
+                for (int u = 0; u < 4; ++u) mx4[u] = fmax3(mx4[u], sv[cix + u], sv[cix + 4 + u]);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mx4[u] = fmaxf(mx4[u], sv[124 + u]);
+            const float mx = fmax3(mx4[0], mx4[1], fmaxf(mx4[2], mx4[3]));
+            const float m_new = fmaxf(m_used, mx * c);
+            const bool need = (m_new > m_used + kF8RescaleThreshold);
+            const bool rescale = __any_sync(0xffffffffu, need);
+            float alpha = 1.f;
+            if (rescale) {
+                alpha = (m_new == -INFINITY) ? 1.f : ex2(m_used - m_new);
+                l *= alpha;
+                m_used = m_new;
+            }
+            const float msub = (m_used == -INFINITY) ? 0.f : m_used;
+            const float2 c2 = make_float2(c, c);
+            const float2 nm2 = make_float2(-msub, -msub);
+            float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+            // P (<= 2^8 with the stale max) as e4m3, four keys per column
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int t = 0; t < 16; ++t) {
+                    const int cix = half * 64 + 4 * t;
+                    const float2 x0 = __ffma2_rn(make_float2(sv[cix], sv[cix + 1]), c2, nm2);
+                    const float2 x1 = __ffma2_rn(make_float2(sv[cix + 2], sv[cix + 3]), c2, nm2);
+                    const float p0 = ex2(x0.x), p1 = ex2(x0.y), p2 = ex2(x1.x), p3 = ex2(x1.y);
+                    ls2[t & 1] = __fadd2_rn(ls2[t & 1], __fadd2_rn(make_float2(p0, p1), make_float2(p2, p3)));
+                    pk[t] = pack_e4m3x4(p0, p1, p2, p3);
+                }
+                tmem_st16(tS + half * 16, pk);
+            }
+            l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
+            if (rescale && j > 0) {
+#pragma unroll 1
+                for (int q = 0; q < kF8D / 32; ++q) {
+                    uint32_t orow[32];
+                    tmem_ld32(tO + q * 32, orow);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int t = 0; t < 32; ++t) orow[t] = __float_as_uint(__uint_as_float(orow[t]) * alpha);
+                    tmem_st32(tO + q * 32, orow);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_full[s]);
+        }
+        if (ok && nkv[s] > 0) {
+            ok = mbar_wait(&o_full[s], 0, abort_flag, kF8O);
+            if (__all_sync(0xffffffffu, ok)) {
+                tc_fence_after();
+                const float out_scale = p.o_scale / l;
+                const bool valid = qrow < p.N;
+                __nv_bfloat16* orow_g =
+                    reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(bh) * p.N + qrow) * kF8D;
+#pragma unroll 1
+                for (int q = 0; q < kF8D / 32; ++q) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + q * 32, ov);
+                    tmem_ld_wait();
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int t = 0; t < 16; ++t)
+                        pk[t] = pack_bf16x2(__uint_as_float(ov[2 * t]) * out_scale,
+                                            __uint_as_float(ov[2 * t + 1]) * out_scale);
+                    if (valid) {
+                        uint4* dst = reinterpret_cast<uint4*>(orow_g + q * 32);
+#pragma unroll
+                        for (int t = 0; t < 4; ++t)
+                            dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+                    }
+                }
+                if (valid) p.lse[static_cast<size_t>(bh) * p.N + qrow] = (m_used + lg2f(l)) * 0.69314718055994531f;
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                           cudaStream_t stream) {
+    const unsigned grid = static_cast<unsigned>(p.n_mblocks) * p.B * p.Hq;
+    if (grid == 0) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(fa_fwd_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, F8Layout::kAlloc);
+    if (e != cudaSuccess) return e;
+    fa_fwd_fp8_kernel<<<grid, kF8Threads, F8Layout::kAlloc, stream>>>(tq, tk, tv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace fa

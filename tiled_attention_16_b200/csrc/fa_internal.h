@@ -23,6 +23,7 @@ struct FwdParams {
     int heads_per_group;
     void* o;           // bf16 [B,Hq,N,D]
     float* lse;        // fp32 [B,Hq,N]
+    float o_scale;     // multiplies O before the 1/l normalisation (FP8: V's descale; 1 for bf16)
 };
 
 struct BwdParams {
@@ -48,6 +49,11 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D);
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, cudaStream_t stream);
+
+// FP8 forward (D = 128): q/k/v maps over e4m3 bytes; p.scale_log2 already
+// includes the Q and K descales, p.o_scale is V's descale.
+cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                           cudaStream_t stream);
 
 // dq_acc == nullptr: do not zero a dQ accumulator (separate dQ pass).
 cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse,

@@ -86,6 +86,31 @@ def make_inputs(wl: Workload):
     return tuple(out)
 
 
+E4M3_MAX = 448.0
+
+
+def make_fp8_inputs(wl: Workload):
+    """FP8 forward inputs for ``wl``: the fp32 draws of ``make_inputs``'s
+    recipe (same generator, seed and order) encoded per tensor as e4m3 with
+    descale = amax / 448, the largest finite e4m3 magnitude.  Returns
+    (q8, k8, v8, q_scale, k_scale, v_scale); element x of q8 stands for
+    float(x) * q_scale."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(wl.seed)
+    shapes = [((wl.B, wl.Hq, wl.N, wl.D), wl.sigma_qk), ((wl.B, wl.Hkv, wl.N, wl.D), wl.sigma_qk),
+              ((wl.B, wl.Hkv, wl.N, wl.D), wl.sigma_vdo)]
+    tens, scales = [], []
+    for shape, sigma in shapes:
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        if sigma != 1.0:
+            x.mul_(sigma)
+        s = float(x.abs().max()) / E4M3_MAX
+        s = s if s > 0 else 1.0
+        tens.append((x / s).to(torch.float8_e4m3fn).contiguous())
+        scales.append(s)
+    return tens[0], tens[1], tens[2], scales[0], scales[1], scales[2]
+
+
 def sample_indices(n: int, count: int, seed: int, must=()):
     """Seeded sorted sample of ``count`` distinct indices in [0, n), always
     including the valid entries of ``must`` (e.g. first/last rows, tile edges)."""
