@@ -8,6 +8,7 @@ from .attention_oracle import (  # noqa: F401
     attention_backward_sampled,
     attention_forward,
     attention_forward_blocked,
+    attention_forward_kv,
     attention_forward_rows,
     attention_rows_fwd_bwd,
     head_row_stats,

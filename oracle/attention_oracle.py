@@ -31,7 +31,9 @@ against the pages by eye:
 
 Conventions: q, do are [B, Hq, N, D]; k, v are [B, Hkv, N, D]; query head h
 reads K/V head h // (Hq // Hkv) (contiguous groups).  Causal means key j is
-visible to query i iff j <= i.  lse is the natural log of the scaled logits.
+visible to query i iff j <= i (for Nq new queries over an Nk-long K/V
+history, attention_forward_kv: iff j <= Nk - Nq + i).  lse is the natural log
+of the scaled logits.
 Parity status: every function here is pinned by tests/test_oracle_pins.py
 (closed forms, invariants, hand-worked golden values, brute force, central
 finite differences and a torch autograd cross-check).
@@ -103,6 +105,37 @@ def attention_forward(q, k, v, scale: float, causal: bool):
         for h in range(Hq):
             g = kv_head_of(h, Hq, Hkv)
             o[b, h], lse[b, h] = _head_forward(q[b, h], k[b, g], v[b, g], scale, causal)
+    return o, lse
+
+
+def attention_forward_kv(q, k, v, scale: float, causal: bool):
+    """Attention of Nq new queries over an Nk-long K/V history (Nq <= Nk).
+
+    This is the incremental computation with a reused KV cache that the
+    Ascend ops-transformer article lists among FlashAttention's suitable cases
+    (section 七, multi-turn dialogue).  The pages fix no mask convention for
+    it; the plainest reading is used: the new queries are the last Nq
+    positions of the sequence, so query i stands at position Nk - Nq + i and,
+    with causal masking, sees keys j <= Nk - Nq + i.  With Nq == Nk this is
+    attention_forward.  q [B, Hq, Nq, D]; k, v [B, Hkv, Nk, D].  Returns
+    (O [B, Hq, Nq, D], LSE [B, Hq, Nq]) in fp64."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if Nq > Nk:
+        raise ValueError("need Nq <= Nk")
+    pos = np.arange(Nq) + (Nk - Nq)  # absolute positions of the queries
+    o = np.empty_like(q)
+    lse = np.empty((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            for c0 in range(0, Nq, _ROW_CHUNK):
+                sl = slice(c0, min(Nq, c0 + _ROW_CHUNK))
+                s = scores(q[b, h, sl], k[b, g], scale, pos[sl], causal)
+                l = row_lse(s)
+                o[b, h, sl] = probs(s, l) @ v[b, g]
+                lse[b, h, sl] = l
     return o, lse
 
 

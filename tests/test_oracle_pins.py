@@ -383,3 +383,71 @@ def test_workload_inputs_are_seeded_bf16():
     assert 2.0 < float(s[0].float().std()) < 4.0 and 0.7 < float(s[2].float().std()) < 1.3
     idx = sample_indices(1000, 10, 3, must=(0, 999))
     assert len(idx) == 10 and 0 in idx and 999 in idx and idx == sorted(idx)
+
+
+# ---------------------------------------------------------------- KV history (Nq <= Nk)
+def _brute_kv(q, k, v, scale, causal):
+    """Scalar loops over plain lists: query i stands at position Nk - Nq + i."""
+    Nq, Nk, D = len(q), len(k), len(k[0])
+    O, L = [], []
+    for i in range(Nq):
+        pos = Nk - Nq + i
+        vis = [j for j in range(Nk) if not (causal and j > pos)]
+        s = {j: scale * sum(q[i][d] * k[j][d] for d in range(D)) for j in vis}
+        z = sum(math.exp(s[j]) for j in vis)
+        O.append([sum(math.exp(s[j]) / z * v[j][d] for j in vis) for d in range(D)])
+        L.append(math.log(z))
+    return O, L
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 9), (3, 7), (7, 7), (2, 13)])
+def test_kv_history_brute_force(causal, Nq, Nk):
+    B, Hq, Hkv, D = 1, 4, 2, 3
+    q = rand((B, Hq, Nq, D), 900 + Nq, 1.5)
+    k = rand((B, Hkv, Nk, D), 901 + Nk, 1.5)
+    v = rand((B, Hkv, Nk, D), 902)
+    o, lse = oracle.attention_forward_kv(q, k, v, 0.7, causal)
+    for h in range(Hq):
+        O, L = _brute_kv(q[0, h].tolist(), k[0, h // 2].tolist(), v[0, h // 2].tolist(), 0.7, causal)
+        np.testing.assert_allclose(o[0, h], O, atol=1e-13)
+        np.testing.assert_allclose(lse[0, h], L, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_kv_history_is_the_suffix_of_full_attention(causal):
+    """Decoding the last Nq queries against the whole K/V gives exactly the last
+    Nq rows of the square computation (the incremental computation reuses the
+    cache instead of recomputing the prefix)."""
+    B, Hq, Hkv, N, D = 2, 4, 1, 300, 16
+    q, k, v, _ = rand_qkv(B, Hq, Hkv, N, D, 910)
+    o_full, lse_full = oracle.attention_forward(q, k, v, 0.25, causal)
+    for Nq in (1, 5, 128, 300):
+        o, lse = oracle.attention_forward_kv(q[:, :, N - Nq:], k, v, 0.25, causal)
+        np.testing.assert_allclose(o, o_full[:, :, N - Nq:], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse, lse_full[:, :, N - Nq:], rtol=0, atol=1e-12)
+
+
+def test_kv_history_zero_queries_average_visible_values():
+    """q = 0: uniform weights over the visible keys, lse = ln(#visible)."""
+    Nq, Nk, D = 4, 10, 3
+    v = rand((1, 1, Nk, D), 920)
+    q = np.zeros((1, 1, Nq, D))
+    k = rand((1, 1, Nk, D), 921)
+    o, lse = oracle.attention_forward_kv(q, k, v, 1.0, True)
+    for i in range(Nq):
+        n_vis = Nk - Nq + i + 1
+        np.testing.assert_allclose(o[0, 0, i], v[0, 0, :n_vis].mean(axis=0), atol=1e-14)
+        assert abs(lse[0, 0, i] - math.log(n_vis)) < 1e-14
+
+
+def test_kv_history_single_query_sees_everything():
+    q = rand((1, 2, 1, 8), 930)
+    k = rand((1, 2, 50, 8), 931)
+    v = rand((1, 2, 50, 8), 932)
+    a = oracle.attention_forward_kv(q, k, v, 0.3, True)
+    b = oracle.attention_forward_kv(q, k, v, 0.3, False)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+    with pytest.raises(ValueError):
+        oracle.attention_forward_kv(rand((1, 1, 5, 2), 1), rand((1, 1, 4, 2), 2), rand((1, 1, 4, 2), 3), 1.0, True)
