@@ -89,6 +89,29 @@ FA_API fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, con
 FA_API fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const void* v,
                      float q_scale, float k_scale, float v_scale, void* o, float* lse, void* stream);
 
+/* Attention of Nq new queries over an Nk-long K/V history (KV-cache reuse in
+ * multi-turn inference, "FlashAttention 在昇腾NPU上到底快在哪", section 七).
+ * The queries are the last Nq positions of the sequence: query i stands at
+ * position Nk - Nq + i and, when causal != 0, sees keys j <= Nk - Nq + i.
+ * Requires 1 <= Nq <= Nk; Hq % Hkv == 0; D = 64 or 128; scale finite, > 0. */
+typedef struct {
+    int B, Hq, Hkv, Nq, Nk, D;
+    float scale;
+    int causal;
+} fa_kv_shape;
+
+/* Bytes of device workspace fa_decode needs (0 if the shape is invalid): the
+ * per-key-range partial outputs and log-sum-exps, fp32. */
+FA_API size_t fa_decode_workspace_bytes(const fa_kv_shape* shape);
+
+/* q [B,Hq,Nq,D], k/v [B,Hkv,Nk,D] bf16 contiguous in; o [B,Hq,Nq,D] bf16 and
+ * lse [B,Hq,Nq] fp32 (natural log) out.  The key axis is split across CTAs;
+ * each writes a partial (O, LSE) to `workspace` (256-byte aligned, at least
+ * fa_decode_workspace_bytes) and a second kernel merges them by the
+ * log-sum-exp rule.  Errors and asynchrony as for fa_bwd. */
+FA_API fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* k, const void* v, void* o,
+                    float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Bytes of device workspace fa_bwd needs for `shape` (0 if the shape is invalid):
  * the per-row statistics (LSE in log2 units and D = rowsum(dO o O), each
  * padded to a multiple of 128 rows) and an fp32 dQ accumulator [B,Hq,N,D]. */
@@ -149,11 +172,12 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * kernel kind k the summed duration total_ms[k] and the launch count
  * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
  * preprocess, 2 fused backward (dK, dV and dQ by fp32 reductions), 3 dQ
- * convert, 4 backward dK/dV kernel, 5 backward dQ kernel, 6 FP8 forward (FA_PROFILE_KINDS;
+ * convert, 4 backward dK/dV kernel, 5 backward dQ kernel, 6 FP8 forward, 7 decode
+ * (split kernel and combine together) (FA_PROFILE_KINDS;
  * fa_bwd uses 1, 4, 5 by default and 1, 2, 3 when the environment variable
  * FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
  * objects; no device memory is allocated. */
-#define FA_PROFILE_KINDS 7
+#define FA_PROFILE_KINDS 8
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

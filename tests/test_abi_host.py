@@ -19,7 +19,7 @@ def test_exports_every_declared_symbol():
     names = A.declared_symbols()
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
                           "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
-                          "fa_bwd_noalloc", "fa_fwd_fp8"}
+                          "fa_bwd_noalloc", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -127,7 +127,7 @@ def test_profile_hooks_without_launches():
     A.profile_begin()
     res = A.profile_end()
     assert set(res) == set(A.PROFILE_KINDS)
-    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 7
+    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 8
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
 
 
@@ -167,3 +167,43 @@ def test_fp8_binding_checks_dtype():
     q = torch.zeros(1, 2, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         A.fwd_fp8(q, q, q)
+
+
+def _kv(**kw):
+    d = dict(B=2, Hq=8, Hkv=2, Nq=3, Nk=1000, D=128, scale=0.1, causal=True)
+    d.update(kw)
+    return A.make_kv_shape(d["B"], d["Hq"], d["Hkv"], d["Nq"], d["Nk"], d["D"], d["scale"], d["causal"])
+
+
+def _dec(shape, ws=P * 16, ws_bytes=1 << 40, ptr=P, **over):
+    args = {n: ptr for n in ("q", "k", "v", "o", "lse")}
+    args.update(over)
+    return A.lib().fa_decode(None if shape is None else ctypes.byref(shape), args["q"], args["k"], args["v"],
+                             args["o"], args["lse"], ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw", [dict(Nq=0), dict(Nk=0), dict(Nq=5, Nk=4), dict(Hq=6, Hkv=4), dict(B=0),
+                                dict(scale=0.0), dict(scale=float("nan"))])
+def test_decode_invalid_shapes(kw):
+    assert _dec(_kv(**kw)) == A.FA_ERR_INVALID_ARG
+    assert A.lib().fa_decode_workspace_bytes(ctypes.byref(_kv(**kw))) == 0
+
+
+def test_decode_host_checks():
+    assert _dec(None) == A.FA_ERR_INVALID_ARG
+    assert _dec(_kv(D=96)) == A.FA_ERR_UNSUPPORTED
+    for which in ("q", "k", "v", "o", "lse"):
+        assert _dec(_kv(), **{which: P + 8}) == A.FA_ERR_INVALID_ARG
+    need = A.lib().fa_decode_workspace_bytes(ctypes.byref(_kv()))
+    assert need > 0 and need % 256 == 0
+    assert _dec(_kv(), ws=0) == A.FA_ERR_INVALID_ARG
+    assert _dec(_kv(), ws=P * 16 + 16) == A.FA_ERR_INVALID_ARG   # not 256-byte aligned
+    assert _dec(_kv(), ws_bytes=need - 1) == A.FA_ERR_INVALID_ARG
+
+
+def test_decode_workspace_covers_partials():
+    # rows x splits x (D + 1) fp32 at least, splits >= 1
+    for kw in (dict(), dict(Nq=1, Nk=1), dict(Nq=16, Nk=70000, B=1, Hq=64, Hkv=8), dict(D=64)):
+        s = _kv(**kw)
+        rows = s.B * s.Hq * s.Nq
+        assert A.lib().fa_decode_workspace_bytes(ctypes.byref(s)) >= rows * (s.D + 1) * 4

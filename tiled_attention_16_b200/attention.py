@@ -28,6 +28,11 @@ class FaShape(ctypes.Structure):
                 ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int)]
 
 
+class FaKvShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int), ("Nq", ctypes.c_int),
+                ("Nk", ctypes.c_int), ("D", ctypes.c_int), ("scale", ctypes.c_float), ("causal", ctypes.c_int)]
+
+
 class FAError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -51,6 +56,11 @@ def lib() -> ctypes.CDLL:
         f32 = ctypes.c_float
         L.fa_fwd_fp8.argtypes = [shp, vp, vp, vp, f32, f32, f32, vp, vp, vp]
         L.fa_fwd_fp8.restype = ctypes.c_int
+        kshp = ctypes.POINTER(FaKvShape)
+        L.fa_decode_workspace_bytes.argtypes = [kshp]
+        L.fa_decode_workspace_bytes.restype = ctypes.c_size_t
+        L.fa_decode.argtypes = [kshp, vp, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.fa_decode.restype = ctypes.c_int
         L.fa_fwd.restype = ctypes.c_int
         L.fa_bwd_workspace_bytes.argtypes = [shp]
         L.fa_bwd_workspace_bytes.restype = sz
@@ -159,6 +169,47 @@ def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_scale: float
     return out, lse
 
 
+def make_kv_shape(B, Hq, Hkv, Nq, Nk, D, scale, causal) -> FaKvShape:
+    return FaKvShape(int(B), int(Hq), int(Hkv), int(Nq), int(Nk), int(D), float(scale), 1 if causal else 0)
+
+
+def decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, D, causal=True, scale=None) -> int:
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    return int(lib().fa_decode_workspace_bytes(ctypes.byref(make_kv_shape(B, Hq, Hkv, Nq, Nk, D, scale, causal))))
+
+
+def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = True, scale: float | None = None,
+           out: torch.Tensor | None = None, lse: torch.Tensor | None = None, workspace: torch.Tensor | None = None):
+    """Attention of Nq new queries q [B,Hq,Nq,D] over an Nk-long K/V history
+    k, v [B,Hkv,Nk,D] (bf16); query i stands at position Nk - Nq + i.
+    Returns (o [B,Hq,Nq,D] bf16, lse [B,Hq,Nq] fp32)."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q and k must be [B, H, N, D]")
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(q, "q", (B, Hq, Nq, D))
+    _check(k, "k", (B, Hkv, Nk, D))
+    _check(v, "v", (B, Hkv, Nk, D))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
+    _check(out, "out", (B, Hq, Nq, D))
+    _check(lse, "lse", (B, Hq, Nq), torch.float32)
+    shp = make_kv_shape(B, Hq, Hkv, Nq, Nk, D, scale, causal)
+    nbytes = int(lib().fa_decode_workspace_bytes(ctypes.byref(shp)))
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), device=q.device, dtype=torch.uint8)
+    if workspace.device.type != "cuda" or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    st = lib().fa_decode(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_decode")
+    return out, lse
+
+
 def workspace_bytes(B, Hq, Hkv, N, D, causal=False, scale=None) -> int:
     scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
     shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
@@ -231,7 +282,7 @@ def timeout_sites() -> int:
 
 
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
-                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel")
+                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode")
 
 
 def profile_begin() -> None:

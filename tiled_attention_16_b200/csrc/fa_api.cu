@@ -36,13 +36,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // 3-D map over a contiguous [BH, N, D] tensor: box = 128 bytes of a row
 // (64 bf16 or 128 e4m3) x 128 rows x 1 head, 128-byte swizzle; rows past N
 // read as zero.
-bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int elem_bytes = 2) {
+bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int elem_bytes = 2, int box_rows = kTileM) {
     auto fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t eb = static_cast<cuuint64_t>(elem_bytes);
     cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * eb, static_cast<cuuint64_t>(N) * D * eb};
-    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(kTileM), 1};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows), 1};
     cuuint32_t estr[3] = {1, 1, 1};
     const CUtensorMapDataType dt = elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUresult r = fn(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -85,6 +85,47 @@ fa_status check_device() {
 }
 
 unsigned int g_last_sites = 0;
+
+// Split-KV plan of fa_decode: 64-key tiles, query rows in blocks of 16 per
+// K/V head, and enough key ranges that ~4 CTAs per SM stream the cache.
+struct DecodePlan {
+    int n_row_blocks, n_splits, tiles_per_split;
+    size_t o_part_off, lse_part_off, total;
+};
+
+fa_status check_kv_shape(const fa_kv_shape* s) {
+    if (!s) return FA_ERR_INVALID_ARG;
+    if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->Nq < 1 || s->Nk < 1 || s->Nq > s->Nk) return FA_ERR_INVALID_ARG;
+    if (s->Hq % s->Hkv != 0) return FA_ERR_INVALID_ARG;
+    if (!std::isfinite(s->scale) || !(s->scale > 0.f)) return FA_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(s->B) * s->Hq * s->Nq;
+    const long long BHkv = static_cast<long long>(s->B) * s->Hkv;
+    const long long row_blocks = (static_cast<long long>(s->Hq / s->Hkv) * s->Nq + 15) / 16;
+    if (rows > 0x7fffffffLL || BHkv > 65535 || row_blocks > 65535) return FA_ERR_INVALID_ARG;
+    if (s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
+    return FA_OK;
+}
+
+DecodePlan decode_plan(const fa_kv_shape& s) {
+    DecodePlan pl;
+    const int R = (s.Hq / s.Hkv) * s.Nq;
+    pl.n_row_blocks = (R + 15) / 16;
+    const int n_tiles = (s.Nk + 63) / 64;
+    const long long pairs = static_cast<long long>(s.B) * s.Hkv * pl.n_row_blocks;
+    const long long target = 4LL * 148;
+    long long splits = (target + pairs - 1) / pairs;
+    if (splits > n_tiles) splits = n_tiles;
+    if (splits > 65535) splits = 65535;
+    if (splits < 1) splits = 1;
+    pl.tiles_per_split = static_cast<int>((n_tiles + splits - 1) / splits);
+    pl.n_splits = (n_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    const size_t rows = static_cast<size_t>(s.B) * s.Hq * s.Nq;
+    pl.o_part_off = 0;
+    pl.lse_part_off = up(rows * pl.n_splits * s.D * 4);
+    pl.total = pl.lse_part_off + up(rows * pl.n_splits * 4);
+    return pl;
+}
 
 constexpr int kNumSMs = 148;
 
@@ -254,6 +295,43 @@ fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const 
     p.o_scale = v_scale;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(6, strm, [&] { return launch_fwd_fp8(tq, tk, tv, p, strm); });
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_decode_workspace_bytes(const fa_kv_shape* shape) {
+    if (check_kv_shape(shape) != FA_OK) return 0;
+    return decode_plan(*shape).total;
+}
+
+fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
+                    void* workspace, size_t workspace_bytes, void* stream) {
+    fa_status st = check_kv_shape(shape);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+    const fa_kv_shape& s = *shape;
+    const DecodePlan pl = decode_plan(s);
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < pl.total)
+        return FA_ERR_INVALID_ARG;
+    if ((st = check_device()) != FA_OK) return st;
+    CUtensorMap tk, tv;
+    if (!make_map(&tk, k, s.B * s.Hkv, s.Nk, s.D, 2, 64) || !make_map(&tv, v, s.B * s.Hkv, s.Nk, s.D, 2, 64))
+        return FA_ERR_CUDA;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    DecodeParams p;
+    p.q = q;
+    p.o = o;
+    p.lse = lse;
+    p.o_part = reinterpret_cast<float*>(wsb + pl.o_part_off);
+    p.lse_part = reinterpret_cast<float*>(wsb + pl.lse_part_off);
+    p.Nq = s.Nq;
+    p.Nk = s.Nk;
+    p.G = s.Hq / s.Hkv;
+    p.causal = s.causal ? 1 : 0;
+    p.n_splits = pl.n_splits;
+    p.tiles_per_split = pl.tiles_per_split;
+    p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed(7, strm, [&] { return launch_decode(s.D, tk, tv, p, pl.n_row_blocks, s.B * s.Hkv, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -41,6 +41,20 @@ struct BwdParams {
     int dq_heads_per_group;  // query heads per scheduling group of the dQ pass
 };
 
+// Attention of Nq new queries over an Nk-long K/V history, split over keys.
+struct DecodeParams {
+    const void* q;     // bf16 [B,Hq,Nq,D]
+    void* o;           // bf16 [B,Hq,Nq,D]
+    float* lse;        // fp32 [B,Hq,Nq]
+    float* o_part;     // fp32 [B*Hq*Nq, n_splits, D]: O / l of each key range
+    float* lse_part;   // fp32 [B*Hq*Nq, n_splits]: LSE of each key range (-inf if empty)
+    int Nq, Nk, G, causal;
+    int n_splits, tiles_per_split;  // 64-key tiles per key range
+    float scale_log2;
+};
+cudaError_t launch_decode(int D, const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& p,
+                          int n_row_blocks, int BHkv, cudaStream_t stream);
+
 // Workspace carve-up for the backward (all offsets 256-byte aligned).
 struct BwdWorkspace {
     size_t lse2_off, dvec_off, dq_off, total;

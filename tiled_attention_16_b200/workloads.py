@@ -86,6 +86,52 @@ def make_inputs(wl: Workload):
     return tuple(out)
 
 
+@dataclass(frozen=True)
+class KvWorkload:
+    """Nq new queries over an Nk-long K/V history (query i at position Nk - Nq + i)."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    D: int
+    causal: bool
+    seed: int
+    sigma_qk: float = 1.0
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    def kv_bytes(self) -> int:
+        """Bytes of the K and V history (bf16), the traffic the work is bound by."""
+        return 2 * 2 * self.B * self.Hkv * self.Nk * self.D
+
+
+# Decoding one token per sequence against a 32K-token cache of a Llama-2-70B
+# shaped layer (64 query heads over 8 K/V heads).
+KV_WORKLOADS = {
+    "decode70b": KvWorkload("decode70b", B=8, Hq=64, Hkv=8, Nq=1, Nk=32768, D=128, causal=True, seed=5),
+}
+
+
+def make_kv_inputs(wl: KvWorkload):
+    """(q [B,Hq,Nq,D], k, v [B,Hkv,Nk,D]) bf16 CPU tensors: fp32 randn drawn in
+    the order q, k, v from one generator seeded with wl.seed, q and k times
+    sigma_qk, rounded to bf16."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(wl.seed)
+    out = []
+    for shape, sigma in (((wl.B, wl.Hq, wl.Nq, wl.D), wl.sigma_qk), ((wl.B, wl.Hkv, wl.Nk, wl.D), wl.sigma_qk),
+                         ((wl.B, wl.Hkv, wl.Nk, wl.D), 1.0)):
+        x = torch.randn(shape, generator=g, dtype=torch.float32)
+        if sigma != 1.0:
+            x.mul_(sigma)
+        out.append(x.to(torch.bfloat16).contiguous())
+    return tuple(out)
+
+
 E4M3_MAX = 448.0
 
 
