@@ -347,6 +347,34 @@ def run_gpu(args, wl):
                                 "launches": n8, "timed_alone": True}
         del q8, k8, v8, o8
 
+    # decode (split-KV) on its own workload: bound by reading the K/V history
+    if not args.no_decode:
+        from tiled_attention_16_b200.workloads import KV_WORKLOADS, make_kv_inputs
+        kwl = KV_WORKLOADS["decode70b"]
+        dq_, dk_, dv_ = (x.to(dev) for x in make_kv_inputs(kwl))
+        dws = torch.empty(A.decode_workspace_bytes(kwl.B, kwl.Hq, kwl.Hkv, kwl.Nq, kwl.Nk, kwl.D, kwl.causal),
+                          device=dev, dtype=torch.uint8)
+        do_ = torch.empty_like(dq_)
+        dlse = torch.empty((kwl.B, kwl.Hq, kwl.Nq), device=dev, dtype=torch.float32)
+        # the whole cache (1 GiB) exceeds L2, so consecutive launches read it from HBM
+        for _ in range(3):
+            A.decode(dq_, dk_, dv_, causal=kwl.causal, out=do_, lse=dlse, workspace=dws)
+        torch.cuda.synchronize()
+        A.profile_begin()
+        for _ in range(20):
+            A.decode(dq_, dk_, dv_, causal=kwl.causal, out=do_, lse=dlse, workspace=dws)
+        td, nd = A.profile_end()["fa_decode"]
+        if A.device_status(dev) != A.FA_OK:
+            raise RuntimeError("device status not OK after decode")
+        d_ms = td / nd
+        gbs = kwl.kv_bytes() / (d_ms * 1e-3) / 1e9
+        breakdown["decode"] = {
+            "workload": f"{kwl.name}: B={kwl.B} Hq={kwl.Hq} Hkv={kwl.Hkv} Nq={kwl.Nq} Nk={kwl.Nk} D={kwl.D} causal",
+            "ms": d_ms, "bound": "hbm", "algorithmic_bytes": kwl.kv_bytes(), "achieved_gbs": gbs,
+            "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
+            "peak_source": f"{peak_src} hbm_gbs", "launches": nd, "timed_alone": True}
+        del dq_, dk_, dv_, dws, do_, dlse
+
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -419,6 +447,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the separate FP8 forward measurement")
+    ap.add_argument("--no-decode", action="store_true", help="skip the separate decode (split-KV) measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
