@@ -96,8 +96,9 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- traffic record
-KERNEL_SOURCES = ("fa_api.cu", "fa_fwd.cu", "fa_bwd.cu", "fa_bwd_split.cu", "sm100.cuh", "fa_internal.h")
-TRAFFIC_SUMMARY = os.path.join(ROOT, "profiles", "dram_traffic_long.md")
+KERNEL_SOURCES = ("fa_api.cu", "fa_fwd.cu", "fa_fwd_fp8.cu", "fa_bwd.cu", "fa_bwd_split.cu", "fa_decode.cu",
+                  "sm100.cuh", "fa_internal.h")
+TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "dram_traffic_*.md")
 
 
 def kernel_source_hash() -> str:
@@ -111,12 +112,22 @@ def kernel_source_hash() -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes (read + write) per launch from the committed ncu summary,
-    or None when there is none for this kernel and workload or it was taken
-    on other kernel sources.  The summary's table rows read
-    `| kernel | workload | source hash | read bytes | write bytes | ... |`."""
-    if not os.path.exists(TRAFFIC_SUMMARY):
-        return None
+    """DRAM bytes (read + write) per launch from the committed ncu summaries
+    (profiles/dram_traffic_*.md), or None when there is none for this kernel
+    and workload or it was taken on other kernel sources.  The summaries'
+    table rows read `| kernel | workload | source hash | read bytes | write bytes | ... |`."""
+    import glob
+    src = kernel_source_hash()
+    for path in sorted(glob.glob(TRAFFIC_GLOB)):
+        with open(path) as f:
+            for line in f:
+                cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+                if len(cells) >= 5 and cells[0] == kernel and cells[1] == workload and cells[2] == src:
+                    try:
+                        return int(cells[3]) + int(cells[4])
+                    except ValueError:
+                        return None
+    return None
     src = kernel_source_hash()
     with open(TRAFFIC_SUMMARY) as f:
         for line in f:
@@ -350,7 +361,7 @@ def run_gpu(args, wl):
     # decode (split-KV) on its own workload: bound by reading the K/V history
     if not args.no_decode:
         from tiled_attention_16_b200.workloads import KV_WORKLOADS, make_kv_inputs
-        kwl = KV_WORKLOADS["decode70b"]
+        kwl = KV_WORKLOADS[args.decode_workload]
         dq_, dk_, dv_ = (x.to(dev) for x in make_kv_inputs(kwl))
         dws = torch.empty(A.decode_workspace_bytes(kwl.B, kwl.Hq, kwl.Hkv, kwl.Nq, kwl.Nk, kwl.D, kwl.causal),
                           device=dev, dtype=torch.uint8)
@@ -371,6 +382,7 @@ def run_gpu(args, wl):
         breakdown["decode"] = {
             "workload": f"{kwl.name}: B={kwl.B} Hq={kwl.Hq} Hkv={kwl.Hkv} Nq={kwl.Nq} Nk={kwl.Nk} D={kwl.D} causal",
             "ms": d_ms, "bound": "hbm", "algorithmic_bytes": kwl.kv_bytes(), "achieved_gbs": gbs,
+            "traffic": recorded_traffic("fa_decode_split_kernel", kwl.name),
             "peak_gbs": peaks["hbm_gbs"], "frac": gbs / peaks["hbm_gbs"],
             "peak_source": f"{peak_src} hbm_gbs", "launches": nd, "timed_alone": True}
         del dq_, dk_, dv_, dws, do_, dlse
@@ -448,6 +460,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the separate FP8 forward measurement")
     ap.add_argument("--no-decode", action="store_true", help="skip the separate decode (split-KV) measurement")
+    ap.add_argument("--decode-workload", default="decode70b", help="KV-history workload of the decode measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

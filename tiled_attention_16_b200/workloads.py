@@ -113,6 +113,8 @@ class KvWorkload:
 # shaped layer (64 query heads over 8 K/V heads).
 KV_WORKLOADS = {
     "decode70b": KvWorkload("decode70b", B=8, Hq=64, Hkv=8, Nq=1, Nk=32768, D=128, causal=True, seed=5),
+    # the same layer with 2 sequences at 16K: 134 MB of history (above L2), for profiling
+    "decode_small": KvWorkload("decode_small", B=2, Hq=64, Hkv=8, Nq=1, Nk=16384, D=128, causal=True, seed=6),
 }
 
 
