@@ -104,7 +104,7 @@ def test_workspace_bytes_formula():
         s = A.make_shape(B, Hq, 1, N, D, 0.1, 0)
         npad = -(-N // 128) * 128
         up = lambda x: -(-x // 256) * 256  # noqa: E731
-        expect = 2 * up(B * Hq * npad * 4) + up(B * Hq * N * D * 4)
+        expect = up(4 * 4) + 2 * up(B * Hq * npad * 4) + up(B * Hq * N * D * 4)  # counters, lse2, D, dQ acc
         assert A.lib().fa_bwd_workspace_bytes(ctypes.byref(s)) == expect
 
 

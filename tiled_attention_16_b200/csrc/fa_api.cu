@@ -392,11 +392,15 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
+    p.sched = reinterpret_cast<unsigned int*>(wsb + ws.sched_off);
+    p.n_units_dkdv = T * s.B * s.Hkv;
+    p.n_units_dq = T * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(1, strm, [&] {
         return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
                                      reinterpret_cast<float*>(wsb + ws.dvec_off), separate ? nullptr : p.dq_acc,
-                                     s.B * s.Hq, s.N, Npad, s.scale, strm);
+                                     s.B * s.Hq, s.N, Npad, s.scale,
+                                     reinterpret_cast<unsigned int*>(wsb + ws.sched_off), strm);
     });
     if (separate) {
         if (e == cudaSuccess) e = timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });

@@ -110,7 +110,10 @@ template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                   const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
-                  float4* __restrict__ dq_acc, size_t dq_vec4, int BH, int N, int Npad, float scale) {
+                  float4* __restrict__ dq_acc, size_t dq_vec4, int BH, int N, int Npad, float scale,
+                  unsigned int* __restrict__ sched) {
+    // work counters of the persistent backward kernels start at zero
+    if (blockIdx.x == 0 && threadIdx.x < kSchedCounters) sched[threadIdx.x] = 0u;
     constexpr int kPer = D / 32;  // elements per lane
     const int lane = threadIdx.x & 31;
     const size_t warp_id = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -572,26 +575,28 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D) {
     const size_t BH = static_cast<size_t>(B) * Hq;
     const size_t Npad = (static_cast<size_t>(N) + kTileM - 1) / kTileM * kTileM;
     BwdWorkspace w;
-    w.lse2_off = 0;
-    w.dvec_off = up(BH * Npad * 4);
+    w.sched_off = 0;
+    w.lse2_off = up(kSchedCounters * 4);
+    w.dvec_off = w.lse2_off + up(BH * Npad * 4);
     w.dq_off = w.dvec_off + up(BH * Npad * 4);
     w.total = w.dq_off + up(BH * static_cast<size_t>(N) * D * 4);
     return w;
 }
 
 cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse, float* lse2, float* dvec,
-                                  float* dq_acc, int BH, int N, int Npad, float scale, cudaStream_t stream) {
+                                  float* dq_acc, int BH, int N, int Npad, float scale, unsigned int* sched,
+                                  cudaStream_t stream) {
     const size_t rows = static_cast<size_t>(BH) * Npad;
     const size_t dq_vec4 = dq_acc ? static_cast<size_t>(BH) * N * D / 4 : 0;
     const int grid = grid_for(rows * 32 > dq_vec4 ? rows * 32 : dq_vec4, 256);
     if (D == 128)
         fa_bwd_preprocess<128><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                          static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec,
-                                                         reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale);
+                                                         reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale, sched);
     else
         fa_bwd_preprocess<64><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                         static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec,
-                                                        reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale);
+                                                        reinterpret_cast<float4*>(dq_acc), dq_vec4, BH, N, Npad, scale, sched);
     return cudaGetLastError();
 }
 

@@ -84,7 +84,7 @@ struct DkdvLayout {
     static constexpr int kLse = kDO + 2 * kTileBytes;
     static constexpr int kDvec = kLse + 2 * kTileN * 4;
     static constexpr int kBar = kDvec + 2 * kTileN * 4;
-    static constexpr int kNumBars = 16;
+    static constexpr int kNumBars = 20;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -100,7 +100,7 @@ struct DqLayout {
     static constexpr int kK = kDO + kTileBytes;      // 2 stages
     static constexpr int kV = kK + 2 * kTileBytes;   // 2 stages
     static constexpr int kBar = kV + 2 * kTileBytes;
-    static constexpr int kNumBars = 16;
+    static constexpr int kNumBars = 18;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -110,6 +110,40 @@ struct DqLayout {
 // ===========================================================================
 // dK / dV
 // ===========================================================================
+// One dK/dV work unit: (batch, K/V head, 128-row key block j).  Units are
+// numbered head group by head group, key block ascending inside a group
+// (heaviest first when causal), then head.
+struct DkdvUnit {
+    int j, bkv, b, hkv, i0, per_head, n_it;
+};
+
+__device__ __forceinline__ DkdvUnit dkdv_unit(const BwdParams& p, int T, int u) {
+    DkdvUnit w;
+    const int BHkv = p.B * p.Hkv;
+    const int grp = u / (p.heads_per_group * T);
+    const int h0 = grp * p.heads_per_group;
+    const int nh = min(p.heads_per_group, BHkv - h0);
+    const int rr = u - grp * p.heads_per_group * T;
+    w.j = rr / nh;
+    w.bkv = h0 + (rr - w.j * nh);
+    w.b = w.bkv / p.Hkv;
+    w.hkv = w.bkv - w.b * p.Hkv;
+    w.i0 = p.causal ? w.j : 0;
+    w.per_head = T - w.i0;
+    w.n_it = (p.Hq / p.Hkv) * w.per_head;
+    return w;
+}
+
+// Persistent: one CTA per SM walks work units.  The first unit of CTA c is
+// c; later ones come from an atomic counter, so the heaviest-first order is
+// served greedily.  The producer fetches each unit id and hands it to the MMA
+// thread and the compute warps through a two-slot ring in shared memory.
+// Every pipeline (Q/dO ring, S/dP/P/dS handshakes) keeps one running
+// iteration count across units; K/V and the dK/dV epilogue go once per unit.
+// While the compute warps store a unit's dK/dV, the producer already loads
+// the next unit's K/V and the MMA thread forms its first S^T and dP^T (the
+// S^T / dP^T blocks are free; the next dV MMA waits for the compute warps'
+// first P^T, which they form only after reading dK/dV out).
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -125,47 +159,39 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint8_t* smem = smem_raw + pad;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
     uint64_t* kv_full = bars + 0;
-    uint64_t* q_full = bars + 1;    // [2]
-    uint64_t* q_empty = bars + 3;   // [2]
-    uint64_t* do_full = bars + 5;   // [2]
-    uint64_t* do_empty = bars + 7;  // [2]
+    uint64_t* q_full = bars + 1;       // [2]
+    uint64_t* q_empty = bars + 3;      // [2]
+    uint64_t* do_full = bars + 5;      // [2]
+    uint64_t* do_empty = bars + 7;     // [2]
     uint64_t* s_full = bars + 9;
     uint64_t* dp_full = bars + 10;
     uint64_t* p_full = bars + 11;
     uint64_t* ds_full = bars + 12;
     uint64_t* dkv_full = bars + 13;
     uint64_t* drain = bars + 14;
+    uint64_t* kv_empty = bars + 15;
+    uint64_t* unit_full = bars + 16;   // [2]
+    uint64_t* unit_empty = bars + 18;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // work unit: head groups; inside a group key block j ascending (heaviest
-    // first when causal), then head
-    const int BHkv = p.B * p.Hkv;
     const int T = (p.N + kTileM - 1) / kTileM;
-    const int tile = static_cast<int>(blockIdx.x);
-    const int grp = tile / (p.heads_per_group * T);
-    const int h0 = grp * p.heads_per_group;
-    const int nh = min(p.heads_per_group, BHkv - h0);
-    const int rr = tile - grp * p.heads_per_group * T;
-    const int j = rr / nh;
-    const int bkv = h0 + (rr - j * nh);
-    const int b = bkv / p.Hkv;
-    const int hkv = bkv - b * p.Hkv;
     const int G = p.Hq / p.Hkv;
-    const int i0 = p.causal ? j : 0;
-    const int per_head = T - i0;
-    const int n_it = G * per_head;
+    const int n_units = p.n_units_dkdv;
 
     if (threadIdx.x == 0) {
         mbar_init(kv_full, 1);
+        mbar_init(kv_empty, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
             mbar_init(&do_full[s], 1);
             mbar_init(&do_empty[s], 1);
+            mbar_init(&unit_full[s], 1);
+            mbar_init(&unit_empty[s], kCompute + 1);
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
@@ -186,6 +212,15 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
 
+    // next unit id for the MMA thread and the compute warps (-1: no more work)
+    auto take_unit = [&](int ui, bool& ok) -> int {
+        const int s = ui & 1;
+        ok = mbar_wait(&unit_full[s], (ui >> 1) & 1, abort_flag, kS1Load);
+        const int u = ok ? unit_id[s] : -1;
+        mbar_arrive(&unit_empty[s]);
+        return u;
+    };
+
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -193,38 +228,55 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
-            mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
-            for (int a = 0; a < D / 64; ++a) {
-                tma_load_3d(smem + L::kK + a * L::kAtomBytes, &tmK, kv_full, a * 64, j * kTileN, bkv);
-                tma_load_3d(smem + L::kV + a * L::kAtomBytes, &tmV, kv_full, a * 64, j * kTileN, bkv);
+            int g = 0;        // query-tile iterations of this CTA so far (all units)
+            int n_q = 0, n_do = 0, n_kv = 0;   // loads issued
+            int ui = 0;       // units of this CTA
+            int u = static_cast<int>(blockIdx.x);
+            bool ok = true;
+            while (ok) {
+                const int s = ui & 1;
+                if (ui >= 2 && !(ok = mbar_wait(&unit_empty[s], ((ui >> 1) - 1) & 1, abort_flag, kS1Empty))) break;
+                unit_id[s] = (u < n_units) ? u : -1;
+                mbar_arrive(&unit_full[s]);
+                if (u >= n_units) break;
+                const DkdvUnit w = dkdv_unit(p, T, u);
+                // K/V of this unit once the previous unit's last S^T and dP^T are done
+                if (ui >= 1 && !(ok = mbar_wait(kv_empty, (ui - 1) & 1, abort_flag, kS1Empty))) break;
+                mbar_arrive_expect_tx(kv_full, 2 * L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a) {
+                    tma_load_3d(smem + L::kK + a * L::kAtomBytes, &tmK, kv_full, a * 64, w.j * kTileN, w.bkv);
+                    tma_load_3d(smem + L::kV + a * L::kAtomBytes, &tmV, kv_full, a * 64, w.j * kTileN, w.bkv);
+                }
+                n_kv = ui + 1;
+                for (int it = 0; ok && it < w.n_it; ++it, ++g) {
+                    const int st = g & 1;
+                    const int gh = it / w.per_head;
+                    const int i = w.i0 + (it - gh * w.per_head);
+                    const int bhq = w.b * p.Hq + w.hkv * G + gh;
+                    if (g >= 2 && !(ok = mbar_wait(&q_empty[st], ((g >> 1) - 1) & 1, abort_flag, kS1Empty))) break;
+                    mbar_arrive_expect_tx(&q_full[st], L::kTileBytes + 2 * kTileM * 4);
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_3d(smem + L::kQ + st * L::kTileBytes + a * L::kAtomBytes, &tmQ, &q_full[st], a * 64,
+                                    i * kTileM, bhq);
+                    const size_t srow = static_cast<size_t>(bhq) * p.Npad + static_cast<size_t>(i) * kTileM;
+                    bulk_load(smem + L::kLse + st * kTileM * 4, p.lse2 + srow, kTileM * 4, &q_full[st]);
+                    bulk_load(smem + L::kDvec + st * kTileM * 4, p.dvec + srow, kTileM * 4, &q_full[st]);
+                    n_q = g + 1;
+                    if (g >= 2 && !(ok = mbar_wait(&do_empty[st], ((g >> 1) - 1) & 1, abort_flag, kS1Empty))) break;
+                    mbar_arrive_expect_tx(&do_full[st], L::kTileBytes);
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_3d(smem + L::kDO + st * L::kTileBytes + a * L::kAtomBytes, &tmDO, &do_full[st],
+                                    a * 64, i * kTileM, bhq);
+                    n_do = g + 1;
+                }
+                if (!ok) break;
+                ++ui;
+                u = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.sched + 0, 1u));
             }
-            int issued_q = 0, issued_do = 0;
-            for (int it = 0; it < n_it; ++it) {
-                const int st = it & 1;
-                const int g = it / per_head;
-                const int i = i0 + (it - g * per_head);
-                const int bhq = b * p.Hq + hkv * G + g;
-                if (it >= 2 && !mbar_wait(&q_empty[st], ((it >> 1) - 1) & 1, abort_flag, kS1Empty)) break;
-                mbar_arrive_expect_tx(&q_full[st], L::kTileBytes + 2 * kTileM * 4);
-                for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kQ + st * L::kTileBytes + a * L::kAtomBytes, &tmQ, &q_full[st], a * 64,
-                                i * kTileM, bhq);
-                const size_t srow = static_cast<size_t>(bhq) * p.Npad + static_cast<size_t>(i) * kTileM;
-                bulk_load(smem + L::kLse + st * kTileM * 4, p.lse2 + srow, kTileM * 4, &q_full[st]);
-                bulk_load(smem + L::kDvec + st * kTileM * 4, p.dvec + srow, kTileM * 4, &q_full[st]);
-                issued_q = it + 1;
-                if (it >= 2 && !mbar_wait(&do_empty[st], ((it >> 1) - 1) & 1, abort_flag, kS1Empty)) break;
-                mbar_arrive_expect_tx(&do_full[st], L::kTileBytes);
-                for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kDO + st * L::kTileBytes + a * L::kAtomBytes, &tmDO, &do_full[st], a * 64,
-                                i * kTileM, bhq);
-                issued_do = it + 1;
-            }
-            wait_drain(kv_full, 0, kS1Drain);
-            for (int it = (issued_q > 2 ? issued_q - 2 : 0); it < issued_q; ++it)
-                wait_drain(&q_full[it & 1], (it >> 1) & 1, kS1Drain);
-            for (int it = (issued_do > 2 ? issued_do - 2 : 0); it < issued_do; ++it)
-                wait_drain(&do_full[it & 1], (it >> 1) & 1, kS1Drain);
+            // no copy may still be landing in shared memory when the CTA leaves
+            if (n_kv > 0) wait_drain(kv_full, (n_kv - 1) & 1, kS1Drain);
+            for (int k = (n_q > 2 ? n_q - 2 : 0); k < n_q; ++k) wait_drain(&q_full[k & 1], (k >> 1) & 1, kS1Drain);
+            for (int k = (n_do > 2 ? n_do - 2 : 0); k < n_do; ++k) wait_drain(&do_full[k & 1], (k >> 1) & 1, kS1Drain);
         }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
@@ -236,60 +288,72 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const uint32_t q_base = smem_u32(smem + L::kQ);
             const uint32_t do_base = smem_u32(smem + L::kDO);
             constexpr uint32_t kAtom = L::kAtomBytes;
-            auto issue_dk = [&](int itp) {
-                const uint32_t qa = q_base + (itp & 1) * L::kTileBytes;
+            // dK += dS^T Q for query-tile iteration gp (global count); first = first of its unit
+            auto issue_dk = [&](int gp, bool first) {
+                const uint32_t qa = q_base + (gp & 1) * L::kTileBytes;
 #pragma unroll
                 for (int kk = 0; kk < kTileM / 16; ++kk)
                     mma_ts(tmem + kColDK, tmem + kColDP + packed_col(kk), sdesc_sw128(qa + kk * 2048, kAtom, 1024),
-                           kIdAcc, (itp > 0 || kk > 0));
-                tc_commit(&q_empty[itp & 1]);
+                           kIdAcc, (!first || kk > 0));
+                tc_commit(&q_empty[gp & 1]);
             };
-            bool ok = mbar_wait(kv_full, 0, abort_flag, kS1Load);
-            for (int it = 0; ok && it < n_it; ++it) {
-                const int st = it & 1;
-                const uint32_t sph = (it >> 1) & 1;
-                const uint32_t ph = it & 1;
-                // S^T = K Q^T (the previous P^T was consumed by dV(it-1), issued earlier)
-                if (!(ok = mbar_wait(&q_full[st], sph, abort_flag, kS1Load))) break;
-                tc_fence_after();
-                const uint32_t qa = q_base + st * L::kTileBytes;
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    mma_ss(tmem + kColS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024), kIdSq,
-                           kk > 0);
-                }
-                tc_commit(s_full);
-                // dK += dS^T Q of the previous query tile (dS^T packed in the dP^T block)
-                if (it > 0) {
-                    if (!(ok = mbar_wait(ds_full, ph ^ 1, abort_flag, kS1Mma))) break;
+            bool ok = true;
+            int g = 0;
+            for (int ui = 0; ok; ++ui) {
+                const int u = take_unit(ui, ok);
+                if (!ok || u < 0) break;
+                const int n_it = dkdv_unit(p, T, u).n_it;
+                if (!(ok = mbar_wait(kv_full, ui & 1, abort_flag, kS1Load))) break;
+                for (int it = 0; it < n_it; ++it) {
+                    const int gi = g + it;
+                    const int st = gi & 1;
+                    const uint32_t sph = (gi >> 1) & 1;
+                    const uint32_t ph = gi & 1;
+                    // S^T = K Q^T (the previous P^T was consumed by dV(it-1), issued earlier)
+                    if (!(ok = mbar_wait(&q_full[st], sph, abort_flag, kS1Load))) break;
                     tc_fence_after();
-                    issue_dk(it - 1);
-                }
-                // dP^T = V dO^T
-                if (!(ok = mbar_wait(&do_full[st], sph, abort_flag, kS1Load))) break;
-                tc_fence_after();
-                const uint32_t da = do_base + st * L::kTileBytes;
+                    const uint32_t qa = q_base + st * L::kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
-                    mma_ss(tmem + kColDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(da + off, 16, 1024), kIdSq,
-                           kk > 0);
-                }
-                tc_commit(dp_full);
-                // dV += P^T dO
-                if (!(ok = mbar_wait(p_full, ph, abort_flag, kS1Mma))) break;
-                tc_fence_after();
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                        mma_ss(tmem + kColS, sdesc_sw128(k_base + off, 16, 1024), sdesc_sw128(qa + off, 16, 1024),
+                               kIdSq, kk > 0);
+                    }
+                    tc_commit(s_full);
+                    // dK += dS^T Q of the previous query tile (dS^T packed in the dP^T block)
+                    if (it > 0) {
+                        if (!(ok = mbar_wait(ds_full, ph ^ 1, abort_flag, kS1Mma))) break;
+                        tc_fence_after();
+                        issue_dk(gi - 1, it == 1);
+                    }
+                    // dP^T = V dO^T
+                    if (!(ok = mbar_wait(&do_full[st], sph, abort_flag, kS1Load))) break;
+                    tc_fence_after();
+                    const uint32_t da = do_base + st * L::kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < kTileM / 16; ++kk)
-                    mma_ts(tmem + kColDV, tmem + kColS + packed_col(kk), sdesc_sw128(da + kk * 2048, kAtom, 1024),
-                           kIdAcc, (it > 0 || kk > 0));
-                tc_commit(&do_empty[st]);
-            }
-            if (ok && n_it > 0 && mbar_wait(ds_full, (n_it - 1) & 1, abort_flag, kS1Mma)) {
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t off = (kk >> 2) * kAtom + (kk & 3) * 32;
+                        mma_ss(tmem + kColDP, sdesc_sw128(v_base + off, 16, 1024), sdesc_sw128(da + off, 16, 1024),
+                               kIdSq, kk > 0);
+                    }
+                    tc_commit(dp_full);
+                    if (it == n_it - 1) tc_commit(kv_empty);   // K and V no longer read by this unit
+                    // dV += P^T dO
+                    if (!(ok = mbar_wait(p_full, ph, abort_flag, kS1Mma))) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < kTileM / 16; ++kk)
+                        mma_ts(tmem + kColDV, tmem + kColS + packed_col(kk), sdesc_sw128(da + kk * 2048, kAtom, 1024),
+                               kIdAcc, (it > 0 || kk > 0));
+                    tc_commit(&do_empty[st]);
+                }
+                if (!ok) break;
+                const int gl = g + n_it - 1;   // last iteration of the unit
+                if (!(ok = mbar_wait(ds_full, gl & 1, abort_flag, kS1Mma))) break;
                 tc_fence_after();
-                issue_dk(n_it - 1);
+                issue_dk(gl, n_it == 1);
                 tc_commit(dkv_full);
+                g += n_it;
             }
             tc_commit(drain);
             wait_drain(drain, 0, kS1Drain);
@@ -299,116 +363,127 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int wg = warp >> 2;
         const int wq = warp & 3;
         const int r = (wq << 5) + lane;  // key row of the block = TMEM lane
-        const int kv = j * kTileN + r;
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
         const int c0 = wg * kCols;       // this group's query columns
         const float c = p.scale_log2;
         const float sc = p.scale;
-        const bool kv_ok = kv < p.N;
-        const bool kv_block_partial = (j + 1) * kTileN > p.N;
         float pv[kCols];
         bool ok = true;
-        for (int it = 0; it < n_it; ++it) {
-            const int st = it & 1;
-            const uint32_t ph = it & 1;
-            const int g = it / per_head;
-            const int i = i0 + (it - g * per_head);
-            const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
-            const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
-            ok = mbar_wait(&q_full[st], (it >> 1) & 1, abort_flag, kS1Compute) &&
-                 mbar_wait(s_full, ph, abort_flag, kS1Compute);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint32_t sr[kCols / 32][32];
+        int g = 0;
+        for (int ui = 0; ok; ++ui) {
+            const int u = take_unit(ui, ok);
+            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
+            const DkdvUnit w = dkdv_unit(p, T, u);
+            const int j = w.j;
+            const int kv = j * kTileN + r;
+            const bool kv_ok = kv < p.N;
+            const bool kv_block_partial = (j + 1) * kTileN > p.N;
+            for (int it = 0; it < w.n_it; ++it) {
+                const int gi = g + it;
+                const int st = gi & 1;
+                const uint32_t ph = gi & 1;
+                const int gh = it / w.per_head;
+                const int i = w.i0 + (it - gh * w.per_head);
+                const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
+                const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
+                ok = mbar_wait(&q_full[st], (gi >> 1) & 1, abort_flag, kS1Compute) &&
+                     mbar_wait(s_full, ph, abort_flag, kS1Compute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                {
+                    uint32_t sr[kCols / 32][32];
 #pragma unroll
-                for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
-                tmem_ld_wait();
-                const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
-                // Masked only on the causal diagonal block and on a partial
-                // last key block (both uniform across the warp); there,
-                // columns q < lo are zero (lo = kCols masks a key row past N).
-                const bool diag = p.causal && (i == j);
-                const float2 c2 = make_float2(c, c);
-                static_for<0, kCols / 2>([&](auto tc) {
-                    constexpr int q = 2 * decltype(tc)::value;
-                    const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
-                    const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
-                    pv[q] = exp2_mixed<q>(x.x);
-                    pv[q + 1] = exp2_mixed<q + 1>(x.y);
-                });
-                if (diag || kv_block_partial) {
-                    const int lo = !kv_ok ? kCols : (diag ? r - c0 : 0);
+                    for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
+                    tmem_ld_wait();
+                    const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                    // Masked only on the causal diagonal block and on a partial
+                    // last key block (both uniform across the warp); there,
+                    // columns q < lo are zero (lo = kCols masks a key row past N).
+                    const bool diag = p.causal && (i == j);
+                    const float2 c2 = make_float2(c, c);
+                    static_for<0, kCols / 2>([&](auto tc) {
+                        constexpr int q = 2 * decltype(tc)::value;
+                        const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
+                        const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
+                        pv[q] = exp2_mixed<q>(x.x);
+                        pv[q + 1] = exp2_mixed<q + 1>(x.y);
+                    });
+                    if (diag || kv_block_partial) {
+                        const int lo = !kv_ok ? kCols : (diag ? r - c0 : 0);
 #pragma unroll
-                    for (int q = 0; q < kCols; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
+                        for (int q = 0; q < kCols; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
+                    }
+#pragma unroll
+                    for (int h = 0; h < kCols / 32; ++h) {
+                        uint32_t pk[16];
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pv[32 * h + 2 * t], pv[32 * h + 2 * t + 1]);
+                        tmem_st16(tmem + lane_off + kColS + c0 + h * 16, pk);
+                    }
+                    tmem_st_wait();
                 }
+                tc_fence_before();
+                mbar_arrive(p_full);
+                ok = mbar_wait(dp_full, ph, abort_flag, kS1Compute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
 #pragma unroll
                 for (int h = 0; h < kCols / 32; ++h) {
-                    uint32_t pk[16];
+                    uint32_t dpr[32];
+                    tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
+                    tmem_ld_wait();
+                    uint32_t wv[16];
+                    const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pv[32 * h + 2 * t], pv[32 * h + 2 * t + 1]);
-                    tmem_st16(tmem + lane_off + kColS + c0 + h * 16, pk);
+                    for (int t = 0; t < 16; ++t) {
+                        // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
+                        const int q0 = h * 32 + 2 * t;
+                        const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
+                        const float2 gd = __ffma2_rn(
+                            make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2,
+                            make_float2(-dv2.x, -dv2.y));
+                        const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
+                        wv[t] = pack_bf16x2(d.x, d.y);
+                    }
+                    // packed over columns this group has already read
+                    tmem_st16(tmem + lane_off + kColDP + c0 + h * 16, wv);
                 }
                 tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(ds_full);
             }
-            tc_fence_before();
-            mbar_arrive(p_full);
-            ok = mbar_wait(dp_full, ph, abort_flag, kS1Compute);
+            if (!ok) break;
+            // ---- epilogue: dV, dK rows of this key block (summed over the group)
+            ok = mbar_wait(dkv_full, ui & 1, abort_flag, kS1Compute);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < kCols / 32; ++h) {
-                uint32_t dpr[32];
-                tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
-                tmem_ld_wait();
-                uint32_t w[16];
-                const float2 sc2 = make_float2(sc, sc);
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
-                    const int q0 = h * 32 + 2 * t;
-                    const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
-                    const float2 g = __ffma2_rn(make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])),
-                                                sc2, make_float2(-dv2.x, -dv2.y));
-                    const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), g);
-                    w[t] = pack_bf16x2(d.x, d.y);
-                }
-                // packed over columns this group has already read
-                tmem_st16(tmem + lane_off + kColDP + c0 + h * 16, w);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(ds_full);
-        }
-        // ---- epilogue: dV, dK rows of this key block (summed over the group)
-        if (ok && n_it > 0) {
-            ok = mbar_wait(dkv_full, 0, abort_flag, kS1Compute);
-            if (__all_sync(0xffffffffu, ok)) {
-                tc_fence_after();
-                const size_t row = static_cast<size_t>(bkv) * p.N + kv;
-                constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
+            const size_t row = static_cast<size_t>(w.bkv) * p.N + kv;
+            constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
 #pragma unroll 1
-                for (int which = 0; which < 2; ++which) {
-                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
-                    __nv_bfloat16* dst_row =
-                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kPer;
+            for (int which = 0; which < 2; ++which) {
+                const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
+                __nv_bfloat16* dst_row =
+                    reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kPer;
 #pragma unroll 1
-                    for (int q = 0; q < kPer / 16; ++q) {
-                        uint32_t v16[16];
-                        tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
-                        tmem_ld_wait();
-                        uint32_t pk[8];
+                for (int q = 0; q < kPer / 16; ++q) {
+                    uint32_t v16[16];
+                    tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
+                    tmem_ld_wait();
+                    uint32_t pk[8];
 #pragma unroll
-                        for (int t = 0; t < 8; ++t)
-                            pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
-                        if (kv_ok) {
-                            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
-                            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-                        }
+                    for (int t = 0; t < 8; ++t)
+                        pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
+                    if (kv_ok) {
+                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
                     }
                 }
             }
+            // the next unit's dV / dK MMAs overwrite these columns only after this
+            // group's next P^T arrival (p_full), which follows these completed loads
+            tc_fence_before();
+            g += w.n_it;
         }
     }
 
@@ -423,6 +498,34 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 // ===========================================================================
 // dQ
 // ===========================================================================
+// One dQ work unit: (batch, query head, 128-row query tile i).  Units are
+// numbered head group by head group, heaviest (last) query tile first inside
+// a group, then head.
+struct DqUnit {
+    int i, bh, kvh, n_j;
+};
+
+__device__ __forceinline__ DqUnit dq_unit(const BwdParams& p, int T, int u) {
+    DqUnit w;
+    const int BH = p.B * p.Hq;
+    const int grp = u / (p.dq_heads_per_group * T);
+    const int h0 = grp * p.dq_heads_per_group;
+    const int nh = min(p.dq_heads_per_group, BH - h0);
+    const int rr = u - grp * p.dq_heads_per_group * T;
+    w.i = T - 1 - rr / nh;
+    w.bh = h0 + (rr % nh);
+    const int b = w.bh / p.Hq;
+    const int h = w.bh - b * p.Hq;
+    w.kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+    w.n_j = p.causal ? w.i + 1 : T;
+    return w;
+}
+
+// Persistent in the same way as the dK/dV kernel: units from an atomic
+// counter, handed over through a two-slot ring; the K/V ring and the S / dP /
+// dS handshakes count key tiles across units.  Q and dO have one buffer: the
+// next unit's tiles load once the current unit's last S and dP have read them
+// (q_empty), while the compute warps store the current dQ.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -437,44 +540,37 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
     uint8_t* smem = smem_raw + pad;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-    uint64_t* q_full = bars + 0;     // Q and dO
-    uint64_t* k_full = bars + 1;     // [2]
-    uint64_t* v_full = bars + 3;     // [2]
-    uint64_t* kv_empty = bars + 5;   // [2]
+    uint64_t* q_full = bars + 0;       // Q and dO
+    uint64_t* k_full = bars + 1;       // [2]
+    uint64_t* v_full = bars + 3;       // [2]
+    uint64_t* kv_empty = bars + 5;     // [2]
     uint64_t* s_full = bars + 7;
     uint64_t* s_free = bars + 8;
     uint64_t* dp_full = bars + 9;
     uint64_t* ds_full = bars + 10;
     uint64_t* dq_done = bars + 11;
     uint64_t* drain = bars + 12;
+    uint64_t* q_empty = bars + 13;
+    uint64_t* unit_full = bars + 14;   // [2]
+    uint64_t* unit_empty = bars + 16;  // [2]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // work unit: head groups; inside a group the heaviest (last) query tiles
-    // first, then the head
-    const int BH = p.B * p.Hq;
     const int T = (p.N + kTileM - 1) / kTileM;
-    const int tile = static_cast<int>(blockIdx.x);
-    const int grp = tile / (p.dq_heads_per_group * T);
-    const int h0 = grp * p.dq_heads_per_group;
-    const int nh = min(p.dq_heads_per_group, BH - h0);
-    const int rr = tile - grp * p.dq_heads_per_group * T;
-    const int i = T - 1 - rr / nh;
-    const int bh = h0 + (rr % nh);
-    const int b = bh / p.Hq;
-    const int h = bh - b * p.Hq;
-    const int kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
-    const int n_j = p.causal ? i + 1 : T;
+    const int n_units = p.n_units_dq;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&k_full[s], 1);
             mbar_init(&v_full[s], 1);
             mbar_init(&kv_empty[s], 1);
+            mbar_init(&unit_full[s], 1);
+            mbar_init(&unit_empty[s], kCompute + 1);
         }
         mbar_init(s_full, 1);
         mbar_init(s_free, kCompute);
@@ -495,6 +591,14 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
 
+    auto take_unit = [&](int ui, bool& ok) -> int {
+        const int s = ui & 1;
+        ok = mbar_wait(&unit_full[s], (ui >> 1) & 1, abort_flag, kS2Load);
+        const int u = ok ? unit_id[s] : -1;
+        mbar_arrive(&unit_empty[s]);
+        return u;
+    };
+
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -502,29 +606,46 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             tma_prefetch_desc(&tmDO);
-            mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
-            for (int a = 0; a < D / 64; ++a) {
-                tma_load_3d(smem + L::kQ + a * L::kAtomBytes, &tmQ, q_full, a * 64, i * kTileM, bh);
-                tma_load_3d(smem + L::kDO + a * L::kAtomBytes, &tmDO, q_full, a * 64, i * kTileM, bh);
+            int gj = 0;               // key tiles of this CTA so far (all units)
+            int n_kv = 0, n_q = 0;    // K/V pairs and Q/dO pairs issued
+            int ui = 0;
+            int u = static_cast<int>(blockIdx.x);
+            bool ok = true;
+            while (ok) {
+                const int s = ui & 1;
+                if (ui >= 2 && !(ok = mbar_wait(&unit_empty[s], ((ui >> 1) - 1) & 1, abort_flag, kS2Load))) break;
+                unit_id[s] = (u < n_units) ? u : -1;
+                mbar_arrive(&unit_full[s]);
+                if (u >= n_units) break;
+                const DqUnit w = dq_unit(p, T, u);
+                if (ui >= 1 && !(ok = mbar_wait(q_empty, (ui - 1) & 1, abort_flag, kS2Load))) break;
+                mbar_arrive_expect_tx(q_full, 2 * L::kTileBytes);
+                for (int a = 0; a < D / 64; ++a) {
+                    tma_load_3d(smem + L::kQ + a * L::kAtomBytes, &tmQ, q_full, a * 64, w.i * kTileM, w.bh);
+                    tma_load_3d(smem + L::kDO + a * L::kAtomBytes, &tmDO, q_full, a * 64, w.i * kTileM, w.bh);
+                }
+                n_q = ui + 1;
+                for (int jj = 0; jj < w.n_j; ++jj, ++gj) {
+                    const int st = gj & 1;
+                    if (gj >= 2 && !(ok = mbar_wait(&kv_empty[st], ((gj >> 1) - 1) & 1, abort_flag, kS2Load))) break;
+                    mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_3d(smem + L::kK + st * L::kTileBytes + a * L::kAtomBytes, &tmK, &k_full[st], a * 64,
+                                    jj * kTileN, w.kvh);
+                    mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
+                    for (int a = 0; a < D / 64; ++a)
+                        tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &v_full[st], a * 64,
+                                    jj * kTileN, w.kvh);
+                    n_kv = gj + 1;
+                }
+                if (!ok) break;
+                ++ui;
+                u = static_cast<int>(gridDim.x) + static_cast<int>(atomicAdd(p.sched + 1, 1u));
             }
-            int issued = 0;
-            for (int jj = 0; jj < n_j; ++jj) {
-                const int st = jj & 1;
-                if (jj >= 2 && !mbar_wait(&kv_empty[st], ((jj >> 1) - 1) & 1, abort_flag, kS2Load)) break;
-                mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
-                for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kK + st * L::kTileBytes + a * L::kAtomBytes, &tmK, &k_full[st], a * 64,
-                                jj * kTileN, kvh);
-                mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
-                for (int a = 0; a < D / 64; ++a)
-                    tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &v_full[st], a * 64,
-                                jj * kTileN, kvh);
-                issued = jj + 1;
-            }
-            wait_drain(q_full, 0, kS2Drain);
-            for (int jj = (issued > 2 ? issued - 2 : 0); jj < issued; ++jj) {
-                wait_drain(&k_full[jj & 1], (jj >> 1) & 1, kS2Drain);
-                wait_drain(&v_full[jj & 1], (jj >> 1) & 1, kS2Drain);
+            if (n_q > 0) wait_drain(q_full, (n_q - 1) & 1, kS2Drain);
+            for (int k = (n_kv > 2 ? n_kv - 2 : 0); k < n_kv; ++k) {
+                wait_drain(&k_full[k & 1], (k >> 1) & 1, kS2Drain);
+                wait_drain(&v_full[k & 1], (k >> 1) & 1, kS2Drain);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -557,43 +678,55 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                 }
                 tc_commit(dp_full);
             };
-            bool ok = mbar_wait(q_full, 0, abort_flag, kS2Load) && mbar_wait(&k_full[0], 0, abort_flag, kS2Load);
-            if (ok) {
+            bool ok = true;
+            int gj = 0;   // key tiles issued (all units)
+            for (int ui = 0; ok; ++ui) {
+                const int u = take_unit(ui, ok);
+                if (!ok || u < 0) break;
+                const int n_j = dq_unit(p, T, u).n_j;
+                // S and dP of the unit's first key tile; the S block is reused once
+                // the compute warps have read the previous S (s_free)
+                if (!(ok = mbar_wait(q_full, ui & 1, abort_flag, kS2Load))) break;
+                if (gj > 0 && !(ok = mbar_wait(s_free, (gj - 1) & 1, abort_flag, kS2Mma))) break;
+                if (!(ok = mbar_wait(&k_full[gj & 1], (gj >> 1) & 1, abort_flag, kS2Load))) break;
                 tc_fence_after();
-                issue_s(0);
-                ok = mbar_wait(&v_full[0], 0, abort_flag, kS2Load);
-                if (ok) {
-                    tc_fence_after();
-                    issue_dp(0);
-                }
-            }
-            for (int jj = 0; ok && jj < n_j; ++jj) {
-                const int st = jj & 1;
-                const uint32_t ph = jj & 1;
-                // S(j+1) once the compute warps have read S(j)
-                if (jj + 1 < n_j) {
-                    if (!(ok = mbar_wait(s_free, ph, abort_flag, kS2Mma))) break;
-                    if (!(ok = mbar_wait(&k_full[st ^ 1], ((jj + 1) >> 1) & 1, abort_flag, kS2Load))) break;
-                    tc_fence_after();
-                    issue_s(st ^ 1);
-                }
-                // dQ += dS K_j (dS packed as bf16 in the dP block)
-                if (!(ok = mbar_wait(ds_full, ph, abort_flag, kS2Mma))) break;
+                issue_s(gj & 1);
+                if (!(ok = mbar_wait(&v_full[gj & 1], (gj >> 1) & 1, abort_flag, kS2Load))) break;
                 tc_fence_after();
-                const uint32_t ka = k_base + st * L::kTileBytes;
+                issue_dp(gj & 1);
+                if (n_j == 1) tc_commit(q_empty);   // Q and dO no longer read by this unit
+                for (int jj = 0; jj < n_j; ++jj) {
+                    const int G = gj + jj;
+                    const int st = G & 1;
+                    const uint32_t ph = G & 1;
+                    // S(j+1) once the compute warps have read S(j)
+                    if (jj + 1 < n_j) {
+                        if (!(ok = mbar_wait(s_free, ph, abort_flag, kS2Mma))) break;
+                        if (!(ok = mbar_wait(&k_full[st ^ 1], ((G + 1) >> 1) & 1, abort_flag, kS2Load))) break;
+                        tc_fence_after();
+                        issue_s(st ^ 1);
+                    }
+                    // dQ += dS K_j (dS packed as bf16 in the dP block)
+                    if (!(ok = mbar_wait(ds_full, ph, abort_flag, kS2Mma))) break;
+                    tc_fence_after();
+                    const uint32_t ka = k_base + st * L::kTileBytes;
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 16; ++kk)
-                    mma_ts(tmem + kColDQ, tmem + kColDP + packed_col(kk), sdesc_sw128(ka + kk * 2048, kAtom, 1024),
-                           kIdDQ, (jj > 0 || kk > 0));
-                tc_commit(&kv_empty[st]);
-                // dP(j+1): its block held dS(j), consumed by the MMAs just issued
-                if (jj + 1 < n_j) {
-                    if (!(ok = mbar_wait(&v_full[st ^ 1], ((jj + 1) >> 1) & 1, abort_flag, kS2Load))) break;
-                    tc_fence_after();
-                    issue_dp(st ^ 1);
+                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                        mma_ts(tmem + kColDQ, tmem + kColDP + packed_col(kk), sdesc_sw128(ka + kk * 2048, kAtom, 1024),
+                               kIdDQ, (jj > 0 || kk > 0));
+                    tc_commit(&kv_empty[st]);
+                    // dP(j+1): its block held dS(j), consumed by the MMAs just issued
+                    if (jj + 1 < n_j) {
+                        if (!(ok = mbar_wait(&v_full[st ^ 1], ((G + 1) >> 1) & 1, abort_flag, kS2Load))) break;
+                        tc_fence_after();
+                        issue_dp(st ^ 1);
+                        if (jj + 2 == n_j) tc_commit(q_empty);
+                    }
                 }
+                if (!ok) break;
+                tc_commit(dq_done);
+                gj += n_j;
             }
-            if (ok) tc_commit(dq_done);
             tc_commit(drain);
             wait_drain(drain, 0, kS2Drain);
         }
@@ -602,98 +735,106 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int wg = warp >> 2;
         const int wq = warp & 3;
         const int r = (wq << 5) + lane;  // query row of the tile = TMEM lane
-        const int qrow = i * kTileM + r;
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
         const int c0 = wg * kCols;       // this group's key columns
         const float c = p.scale_log2;
-        const size_t srow = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(qrow);
-        const float lse2 = p.lse2[srow];   // +inf on padding rows -> P = 0
-        const float dval = p.dvec[srow];   // scale * D
         const float sc = p.scale;
         float pv[kCols];
         bool ok = true;
-        for (int jj = 0; jj < n_j; ++jj) {
-            const uint32_t ph = jj & 1;
-            ok = mbar_wait(s_full, ph, abort_flag, kS2Compute);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            {
-                uint32_t sr[kCols / 32][32];
-#pragma unroll
-                for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
-                tmem_ld_wait();
-                tc_fence_before();
-                mbar_arrive(s_free);
-                const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
-                const int kv0 = jj * kTileN + c0;
-                // Masked only on the causal diagonal tile and on a partial last
-                // key tile (uniform across the warp): key columns t >= hi are
-                // zero (past N, or after this query row on the diagonal).
-                const bool diag = p.causal && jj == i;
-                const float2 c2 = make_float2(c, c);
-                const float2 nl2 = make_float2(-lse2, -lse2);
-                static_for<0, kCols / 2>([&](auto tc) {
-                    constexpr int t = 2 * decltype(tc)::value;
-                    const float2 x = __ffma2_rn(make_float2(sv[t], sv[t + 1]), c2, nl2);
-                    pv[t] = exp2_mixed<t>(x.x);
-                    pv[t + 1] = exp2_mixed<t + 1>(x.y);
-                });
-                if (diag || kv0 + kCols > p.N) {
-                    const int hi = min(p.N, diag ? qrow + 1 : p.N) - kv0;
-#pragma unroll
-                    for (int t = 0; t < kCols; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
-                }
-            }
-            ok = mbar_wait(dp_full, ph, abort_flag, kS2Compute);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int hh = 0; hh < kCols / 32; ++hh) {
-                uint32_t dpr[32];
-                tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
-                tmem_ld_wait();
-                uint32_t w[16];
-                const float2 sc2 = make_float2(sc, sc);
-                const float2 nd2 = make_float2(-dval, -dval);
-#pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dval = scale*D
-                    const int q0 = hh * 32 + 2 * t;
-                    const float2 g = __ffma2_rn(make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])),
-                                                sc2, nd2);
-                    const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), g);
-                    w[t] = pack_bf16x2(d.x, d.y);
-                }
-                tmem_st16(tmem + lane_off + kColDP + c0 + hh * 16, w);
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(ds_full);
-        }
-        // ---- epilogue: dQ rows (already scaled) -> bf16
-        if (ok && n_j > 0) {
-            ok = mbar_wait(dq_done, 0, abort_flag, kS2Compute);
-            if (__all_sync(0xffffffffu, ok)) {
+        int gj = 0;
+        for (int ui = 0; ok; ++ui) {
+            const int u = take_unit(ui, ok);
+            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
+            const DqUnit w = dq_unit(p, T, u);
+            const int i = w.i;
+            const int qrow = i * kTileM + r;
+            const size_t srow = static_cast<size_t>(w.bh) * p.Npad + static_cast<size_t>(qrow);
+            const float lse2 = p.lse2[srow];   // +inf on padding rows -> P = 0
+            const float dval = p.dvec[srow];   // scale * D
+            for (int jj = 0; jj < w.n_j; ++jj) {
+                const uint32_t ph = (gj + jj) & 1;
+                ok = mbar_wait(s_full, ph, abort_flag, kS2Compute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
-                constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
-                __nv_bfloat16* dst_row =
-                    reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(bh) * p.N + qrow) * D + wg * kPer;
-#pragma unroll 1
-                for (int q = 0; q < kPer / 16; ++q) {
-                    uint32_t v16[16];
-                    tmem_ld16(tmem + lane_off + kColDQ + wg * kPer + q * 16, v16);
-                    tmem_ld_wait();
-                    uint32_t pk[8];
+                {
+                    uint32_t sr[kCols / 32][32];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
-                    if (qrow < p.N) {
-                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                    for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    mbar_arrive(s_free);
+                    const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                    const int kv0 = jj * kTileN + c0;
+                    // Masked only on the causal diagonal tile and on a partial last
+                    // key tile (uniform across the warp): key columns t >= hi are
+                    // zero (past N, or after this query row on the diagonal).
+                    const bool diag = p.causal && jj == i;
+                    const float2 c2 = make_float2(c, c);
+                    const float2 nl2 = make_float2(-lse2, -lse2);
+                    static_for<0, kCols / 2>([&](auto tc) {
+                        constexpr int t = 2 * decltype(tc)::value;
+                        const float2 x = __ffma2_rn(make_float2(sv[t], sv[t + 1]), c2, nl2);
+                        pv[t] = exp2_mixed<t>(x.x);
+                        pv[t + 1] = exp2_mixed<t + 1>(x.y);
+                    });
+                    if (diag || kv0 + kCols > p.N) {
+                        const int hi = min(p.N, diag ? qrow + 1 : p.N) - kv0;
+#pragma unroll
+                        for (int t = 0; t < kCols; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
                     }
                 }
+                ok = mbar_wait(dp_full, ph, abort_flag, kS2Compute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int hh = 0; hh < kCols / 32; ++hh) {
+                    uint32_t dpr[32];
+                    tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
+                    tmem_ld_wait();
+                    uint32_t wv[16];
+                    const float2 sc2 = make_float2(sc, sc);
+                    const float2 nd2 = make_float2(-dval, -dval);
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dval = scale*D
+                        const int q0 = hh * 32 + 2 * t;
+                        const float2 gd = __ffma2_rn(
+                            make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2, nd2);
+                        const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
+                        wv[t] = pack_bf16x2(d.x, d.y);
+                    }
+                    tmem_st16(tmem + lane_off + kColDP + c0 + hh * 16, wv);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(ds_full);
             }
+            if (!ok) break;
+            // ---- epilogue: dQ rows (already scaled) -> bf16; the next unit's first
+            // dQ MMA overwrites these columns only after this thread's next ds_full
+            ok = mbar_wait(dq_done, ui & 1, abort_flag, kS2Compute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
+            __nv_bfloat16* dst_row =
+                reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(w.bh) * p.N + qrow) * D + wg * kPer;
+#pragma unroll 1
+            for (int q = 0; q < kPer / 16; ++q) {
+                uint32_t v16[16];
+                tmem_ld16(tmem + lane_off + kColDQ + wg * kPer + q * 16, v16);
+                tmem_ld_wait();
+                uint32_t pk[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
+                if (qrow < p.N) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            tc_fence_before();
+            gj += w.n_j;
         }
     }
 
@@ -703,6 +844,19 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tc_fence_after();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Multiprocessor count of the current device (cached per device).
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+        cache[dev] = n;
+    }
+    return cache[dev];
 }
 
 template <class Kern>
@@ -719,14 +873,20 @@ cudaError_t launch(Kern kern, unsigned grid, int smem, const CUtensorMap& tq, co
 
 cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
-    const unsigned grid = static_cast<unsigned>((p.N + kTileN - 1) / kTileN) * p.B * p.Hkv;
+    // persistent: one CTA per SM walks the units
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    // (with fewer than two units per SM the hardware's own CTA dispatch is as good)
+    const unsigned grid = static_cast<unsigned>(p.n_units_dkdv < 2 * sms ? p.n_units_dkdv : sms);
     if (D == 128) return launch(fa_bwd_dkdv_kernel<128>, grid, DkdvLayout<128>::kAlloc, tq, tk, tv, tdo, p, stream);
     return launch(fa_bwd_dkdv_kernel<64>, grid, DkdvLayout<64>::kAlloc, tq, tk, tv, tdo, p, stream);
 }
 
 cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {
-    const unsigned grid = static_cast<unsigned>((p.N + kTileM - 1) / kTileM) * p.B * p.Hq;
+    const int sms = sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const unsigned grid = static_cast<unsigned>(p.n_units_dq < 2 * sms ? p.n_units_dq : sms);
     if (D == 128) return launch(fa_bwd_dq_kernel<128>, grid, DqLayout<128>::kAlloc, tq, tk, tv, tdo, p, stream);
     return launch(fa_bwd_dq_kernel<64>, grid, DqLayout<64>::kAlloc, tq, tk, tv, tdo, p, stream);
 }

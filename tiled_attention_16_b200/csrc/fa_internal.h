@@ -39,7 +39,13 @@ struct BwdParams {
     void* dk;          // bf16 [B,Hkv,N,D]
     void* dv;          // bf16 [B,Hkv,N,D]
     int dq_heads_per_group;  // query heads per scheduling group of the dQ pass
+    unsigned int* sched;     // work counters of the persistent kernels (zeroed by the preprocess)
+    int n_units_dkdv;        // work units of the dK/dV pass
+    int n_units_dq;          // work units of the dQ pass
 };
+
+// Counters at the start of the backward workspace: [0] dK/dV pass, [1] dQ pass.
+constexpr int kSchedCounters = 4;
 
 // Attention of Nq new queries over an Nk-long K/V history, split over keys.
 struct DecodeParams {
@@ -57,7 +63,7 @@ cudaError_t launch_decode(int D, const CUtensorMap& tk, const CUtensorMap& tv, c
 
 // Workspace carve-up for the backward (all offsets 256-byte aligned).
 struct BwdWorkspace {
-    size_t lse2_off, dvec_off, dq_off, total;
+    size_t sched_off, lse2_off, dvec_off, dq_off, total;
 };
 BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D);
 
@@ -72,7 +78,8 @@ cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const C
 // dq_acc == nullptr: do not zero a dQ accumulator (separate dQ pass).
 cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const float* lse,
                                   float* lse2, float* dvec, float* dq_acc,
-                                  int BH, int N, int Npad, float scale, cudaStream_t stream);
+                                  int BH, int N, int Npad, float scale, unsigned int* sched,
+                                  cudaStream_t stream);
 
 // Fused backward: dK, dV and dQ (fp32 reductions into p.dq_acc).
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
