@@ -86,6 +86,22 @@ fa_status check_device() {
 
 unsigned int g_last_sites = 0;
 
+}  // namespace
+
+int sm_count() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+namespace {
+
 // Split-KV plan of fa_decode: 64-key tiles, query rows in blocks of 16 per
 // K/V head, and enough key ranges that ~4 CTAs per SM stream the cache.
 struct DecodePlan {
@@ -147,6 +163,28 @@ bool dq_separate_mode() {
 // code this name only stands in for the symbol; the device address comes from
 // cudaGetSymbolAddress (noalloc_scratch below).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
+// Work-counter slots of the persistent forward.  Each launch takes the next
+// slot (round robin), so launches that may overlap on different streams use
+// different counters; the last CTA of a launch puts its slot back to zero.
+constexpr int kFwdSchedSlots = 1024;
+static __device__ unsigned int g_fwd_sched[kFwdSchedSlots][2];
+
+fa_status fwd_sched_slot(unsigned int** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    static std::mutex mu;
+    static unsigned int* base[64] = {};
+    static unsigned int next[64] = {};
+    std::lock_guard<std::mutex> g(mu);
+    if (base[dev] == nullptr) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_fwd_sched) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
+        base[dev] = static_cast<unsigned int*>(ptr);
+    }
+    *out = base[dev] + 2 * (next[dev]++ % kFwdSchedSlots);
+    return FA_OK;
+}
 
 // Device address of g_noalloc_scratch on the current device, looked up once
 // per device (with that device current) and cached.
@@ -257,6 +295,8 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.o = o;
     p.lse = lse;
     p.o_scale = 1.f;
+    p.n_units = p.n_mblocks * s.B * s.Hq;
+    if ((st = fwd_sched_slot(&p.sched)) != FA_OK) return st;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -293,6 +333,8 @@ fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const 
     p.o = o;
     p.lse = lse;
     p.o_scale = v_scale;
+    p.n_units = p.n_mblocks * s.B * s.Hq;
+    p.sched = nullptr;  // the FP8 kernel is not persistent
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(6, strm, [&] { return launch_fwd_fp8(tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

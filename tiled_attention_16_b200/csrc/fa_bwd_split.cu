@@ -846,19 +846,6 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
 }
 
-// Multiprocessor count of the current device (cached per device).
-int sm_count() {
-    static int cache[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-    if (cache[dev] == 0) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return -1;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
 template <class Kern>
 cudaError_t launch(Kern kern, unsigned grid, int smem, const CUtensorMap& tq, const CUtensorMap& tk,
                    const CUtensorMap& tv, const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream) {

@@ -24,7 +24,12 @@ struct FwdParams {
     void* o;           // bf16 [B,Hq,N,D]
     float* lse;        // fp32 [B,Hq,N]
     float o_scale;     // multiplies O before the 1/l normalisation (FP8: V's descale; 1 for bf16)
+    int n_units;       // work units: B * Hq * n_mblocks
+    unsigned int* sched;  // [2] counter slot of the persistent forward: next unit, CTAs done
 };
+
+// Multiprocessor count of the current device (cached per device; -1 on error).
+int sm_count();
 
 struct BwdParams {
     int B, Hq, Hkv, N, Npad;
