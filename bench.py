@@ -96,16 +96,25 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- traffic record
-KERNEL_SOURCES = ("fa_api.cu", "fa_fwd.cu", "fa_fwd_fp8.cu", "fa_bwd.cu", "fa_bwd_split.cu", "fa_decode.cu",
-                  "sm100.cuh", "fa_internal.h")
+# Sources that decide what each kernel reads and writes: its own file plus
+# the launch configuration (API layer) and the shared headers.
+COMMON_SOURCES = ("fa_api.cu", "sm100.cuh", "fa_internal.h")
+KERNEL_FILES = {
+    "fa_fwd_kernel": ("fa_fwd.cu",),
+    "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu",),
+    "fa_bwd_dkdv_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
+    "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
+    "fa_bwd_kernel": ("fa_bwd.cu",),
+    "fa_decode_split_kernel": ("fa_decode.cu",),
+    "fa_decode_combine_kernel": ("fa_decode.cu",),
+}
 TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "dram_traffic_*.md")
 
 
-def kernel_source_hash() -> str:
-    """Hash of every source that decides what the kernels read and write
-    (the kernels and the launch configuration chosen by the API layer)."""
+def kernel_source_hash(kernel: str) -> str:
+    """sha256 prefix over the sources of `kernel` (its file and the common ones)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_FILES.get(kernel, ()) + COMMON_SOURCES:
         with open(os.path.join(ROOT, "tiled_attention_16_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -117,7 +126,7 @@ def recorded_traffic(kernel: str, workload: str):
     and workload or it was taken on other kernel sources.  The summaries'
     table rows read `| kernel | workload | source hash | read bytes | write bytes | ... |`."""
     import glob
-    src = kernel_source_hash()
+    src = kernel_source_hash(kernel)
     for path in sorted(glob.glob(TRAFFIC_GLOB)):
         with open(path) as f:
             for line in f:
@@ -127,16 +136,6 @@ def recorded_traffic(kernel: str, workload: str):
                         return int(cells[3]) + int(cells[4])
                     except ValueError:
                         return None
-    return None
-    src = kernel_source_hash()
-    with open(TRAFFIC_SUMMARY) as f:
-        for line in f:
-            cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 5 and cells[0] == kernel and cells[1] == workload and cells[2] == src:
-                try:
-                    return int(cells[3]) + int(cells[4])
-                except ValueError:
-                    return None
     return None
 
 

@@ -207,3 +207,27 @@ def test_lse_consistent_with_output_scale():
     # causal row 0 sees one key: lse_0 = scale * q_0 . k_0
     ref0 = (q[..., 0, :].double() * k[..., 0, :].double()).sum(-1) / math.sqrt(D)
     assert torch.allclose(lse[..., 0].double().cpu(), ref0, atol=1e-3)
+
+
+def test_forward_counter_slots_reused_and_concurrent():
+    """The persistent forward takes a work-counter slot per launch (1024 slots,
+    round robin) and its last CTA resets it: after more than 1024 launches,
+    and with launches interleaved on two streams, results stay bitwise equal."""
+    dev = _gpu()
+    wl = WORKLOADS["tiny"].with_(causal=True, N=700, Hq=4, Hkv=2, D=128)
+    q, k, v, _ = (x.to(dev) for x in make_inputs(wl))
+    o_ref, lse_ref = A.fwd(q, k, v, causal=True)
+    o, lse = torch.empty_like(o_ref), torch.empty_like(lse_ref)
+    for _ in range(1100):
+        A.fwd(q, k, v, causal=True, out=o, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_ref) and torch.equal(lse, lse_ref)
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    outs = [(torch.empty_like(o_ref), torch.empty_like(lse_ref)) for _ in range(8)]
+    for n, (oo, ll) in enumerate(outs):
+        with torch.cuda.stream(s1 if n % 2 == 0 else s2):
+            A.fwd(q, k, v, causal=True, out=oo, lse=ll)
+    torch.cuda.synchronize()
+    assert A.device_status(dev) == A.FA_OK
+    for oo, ll in outs:
+        assert torch.equal(oo, o_ref) and torch.equal(ll, lse_ref)
