@@ -334,7 +334,7 @@ fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const 
     p.lse = lse;
     p.o_scale = v_scale;
     p.n_units = p.n_mblocks * s.B * s.Hq;
-    p.sched = nullptr;  // the FP8 kernel is not persistent
+    if ((st = fwd_sched_slot(&p.sched)) != FA_OK) return st;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(6, strm, [&] { return launch_fwd_fp8(tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
