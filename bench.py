@@ -354,7 +354,8 @@ def run_gpu(args, wl):
         breakdown["fp8_fwd"] = {"ms": f8_ms, "tflops": f8_tf, "peak": 2 * peak_tf,
                                 "frac_of_peak": f8_tf / (2 * peak_tf),
                                 "peak_source": f"{peak_src} bf16_tflops (burst) x 2 (nominal e4m3/bf16 ratio)",
-                                "launches": n8, "timed_alone": True}
+                                "launches": n8, "timed_alone": True,
+                                "traffic": recorded_traffic("fa_fwd_fp8_kernel", wl.name)}
         del q8, k8, v8, o8
 
     # decode (split-KV) on its own workload: bound by reading the K/V history
