@@ -5,14 +5,17 @@ the CUDA library never imports it.
 """
 from .attention_oracle import (  # noqa: F401
     attention_backward,
+    attention_backward_block,
     attention_backward_sampled,
     attention_forward,
+    attention_forward_block,
     attention_forward_blocked,
     attention_forward_kv,
     attention_forward_rows,
     attention_rows_fwd_bwd,
     head_row_stats,
     kv_head_of,
+    merge_partials,
     probs,
     row_lse,
     scores,

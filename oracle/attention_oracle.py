@@ -299,3 +299,110 @@ def attention_forward_blocked(q, k, v, scale: float, causal: bool, block_r: int 
                 o[b, h, rows] = acc / l[:, None]
                 lse[b, h, rows] = m + np.log(l)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Sequence-sharded attention (FlashAttention glossary, section 3.2 "FlashAttention
+# v2改进", item 2 "序列并行"): the sequence is split across devices and each
+# device works on its part.  The page says the per-device attention results
+# are summed (AllReduce); a plain sum of the per-shard outputs is not the
+# attention of the whole sequence.  What is exact is the log-sum-exp merge
+# below: a shard's result over a block of keys is the softmax restricted to
+# those keys, and re-weighting each by the share of the row's total exp-mass
+# that falls in its block gives the full softmax.  The functions here are that
+# definition written out for one key block at a time; positions are absolute
+# (q_off, k_off), so causal masking compares the rows' and keys' places in the
+# whole sequence.
+
+
+def _block_mask(n_q: int, n_k: int, q_off: int, k_off: int, causal: bool) -> np.ndarray:
+    """visible[i, j]: key k_off + j may be seen by query q_off + i."""
+    if not causal:
+        return np.ones((n_q, n_k), dtype=bool)
+    return (np.arange(n_k)[None, :] + k_off) <= (np.arange(n_q)[:, None] + q_off)
+
+
+def attention_forward_block(q, k, v, scale: float, causal: bool, q_off: int = 0, k_off: int = 0):
+    """Attention of the queries q (absolute positions q_off ...) over ONE block
+    of keys k, v (positions k_off ...), normalised over that block only.
+
+    Returns (O_part [B,Hq,Nq,D], LSE_part [B,Hq,Nq]) in fp64 with
+    LSE_part_i = log sum_{j in block, visible} exp(s_ij) and
+    O_part_i = sum_j exp(s_ij - LSE_part_i) v_j.  A row that sees no key of
+    the block gets O_part = 0 and LSE_part = -inf (it carries no mass)."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    vis = _block_mask(Nq, Nk, q_off, k_off, causal)
+    o = np.zeros_like(q)
+    lse = np.full((B, Hq, Nq), -np.inf)
+    seen = vis.any(axis=1)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            for c0 in range(0, Nq, _ROW_CHUNK):
+                sl = slice(c0, min(Nq, c0 + _ROW_CHUNK))
+                rows = np.nonzero(seen[sl])[0] + c0
+                if len(rows) == 0:
+                    continue
+                s = scale * (q[b, h, rows] @ k[b, g].T)
+                s = np.where(vis[rows], s, -np.inf)
+                l = row_lse(s)
+                o[b, h, rows] = probs(s, l) @ v[b, g]
+                lse[b, h, rows] = l
+    return o, lse
+
+
+def merge_partials(o_parts, lse_parts):
+    """Combine the partial results of disjoint key blocks into the result over
+    their union:  LSE = log sum_r exp(LSE_r),  O = sum_r exp(LSE_r - LSE) O_r.
+
+    o_parts: sequence of [..., D] arrays; lse_parts: matching [...] arrays.
+    Rows whose every part is -inf stay O = 0, LSE = -inf."""
+    lse_stack = np.stack([_f64(x) for x in lse_parts])
+    o_stack = np.stack([_f64(x) for x in o_parts])
+    m = lse_stack.max(axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w_raw = np.exp(lse_stack - m_safe[None])          # 0 for -inf parts
+    total = w_raw.sum(axis=0)
+    lse = np.where(total > 0, m_safe + np.log(np.where(total > 0, total, 1.0)), -np.inf)
+    w = np.where(total[None] > 0, w_raw / np.where(total > 0, total, 1.0)[None], 0.0)
+    o = (w[..., None] * o_stack).sum(axis=0)
+    return o, lse
+
+
+def attention_backward_block(q, k, v, o, do, lse, scale: float, causal: bool, q_off: int = 0, k_off: int = 0):
+    """Gradient terms of L = <O, dO> that involve ONE block of keys, given the
+    whole rows' statistics: o (the full attention output) and lse (the full
+    log-sum-exp), as the recomputation of the deep dive's section 改进1 uses
+    them.  With p_ij = exp(s_ij - lse_i) over the block's visible keys:
+        dV_j = sum_i p_ij dO_i,   dP_ij = dO_i . v_j,   D_i = dO_i . o_i,
+        dS_ij = p_ij (dP_ij - D_i),
+        dQ_i^(block) = scale sum_{j in block} dS_ij k_j,   dK_j = scale sum_i dS_ij q_i.
+    D_i = dO_i . o_i equals sum over ALL keys of p_ij dP_ij because
+    o_i = sum_j p_ij v_j.  Summing dQ^(block) over a partition of the keys gives
+    dQ; dK, dV of a key come from its own block alone (summed over the query
+    blocks and over a GQA group's query heads).
+    Returns (dQ_part [B,Hq,Nq,D], dK [B,Hkv,Nk,D], dV [B,Hkv,Nk,D]) in fp64."""
+    q, k, v, o, do, lse = _f64(q), _f64(k), _f64(v), _f64(o), _f64(do), _f64(lse)
+    B, Hq, Nq, D = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    vis = _block_mask(Nq, Nk, q_off, k_off, causal)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            g = kv_head_of(h, Hq, Hkv)
+            kh, vh = k[b, g], v[b, g]
+            for c0 in range(0, Nq, _ROW_CHUNK):
+                r = np.arange(c0, min(Nq, c0 + _ROW_CHUNK))
+                s = np.where(vis[r], scale * (q[b, h, r] @ kh.T), -np.inf)
+                p = np.exp(s - lse[b, h, r][:, None])
+                dp = do[b, h, r] @ vh.T
+                Di = (do[b, h, r] * o[b, h, r]).sum(axis=1)
+                ds = p * (dp - Di[:, None])
+                dq[b, h, r] = scale * (ds @ kh)
+                dk[b, g] += scale * (ds.T @ q[b, h, r])
+                dv[b, g] += p.T @ do[b, h, r]
+    return dq, dk, dv
