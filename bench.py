@@ -387,6 +387,47 @@ def run_gpu(args, wl):
             "peak_source": f"{peak_src} hbm_gbs", "launches": nd, "timed_alone": True}
         del dq_, dk_, dv_, dws, do_, dlse
 
+    # context parallel: the ring of CP_RANKS ranks over this workload's sequence
+    # (zigzag chunks), all ranks' pairs run on this one GPU in ring order; the
+    # exchange is not timed (it needs more GPUs).  Same flop convention as
+    # the step, so the ratio to the step's rate is the chunking's cost.
+    if not args.no_cp and wl.N % (2 * args.cp_ranks) == 0:
+        from tiled_attention_16_b200 import context_parallel as cp
+        R = args.cp_ranks
+        sh = lambda x: [cp.shard_sequence(x, r, R) for r in range(R)]  # noqa: E731
+        cq, ck, cv, cdo = sh(q), sh(k), sh(v), sh(do)
+
+        def ring_step():
+            fw = cp.virtual_ring_fwd(cq, ck, cv, wl.causal, wl.softmax_scale)
+            cp.virtual_ring_bwd(cq, ck, cv, [f[0] for f in fw], cdo, [f[1] for f in fw], wl.causal,
+                                wl.softmax_scale)
+
+        for _ in range(3):
+            ring_step()
+        torch.cuda.synchronize()
+        A.profile_begin()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        n_cp = 5
+        for _ in range(n_cp):
+            ring_step()
+        e1.record()
+        torch.cuda.synchronize()
+        cp_kernels = A.profile_end()
+        if A.device_status(dev) != A.FA_OK:
+            raise RuntimeError("device status not OK after the context-parallel ring")
+        cp_ms = e0.elapsed_time(e1) / n_cp
+        cp_tf = flops_step / (cp_ms * 1e-3) / 1e12
+        step_tf = flops_step / (ms * 1e-3) / 1e12
+        breakdown["context_parallel"] = {
+            "ranks": R, "chunk_rows": wl.N // (2 * R), "layout": "zigzag", "ms_per_step": cp_ms,
+            "tflops": cp_tf, "vs_step_rate": cp_tf / step_tf if step_tf else None,
+            "merge_ms": cp_kernels["fa_lse_merge_kernel"][0] / n_cp,
+            "accumulate_ms": cp_kernels["fa_accumulate_kernel"][0] / n_cp,
+            "launches_per_step": sum(nn for _, nn in cp_kernels.values()) / n_cp,
+            "exchange": "not timed (one GPU): the ranks run one after another on it", "timed_alone": True}
+        del cq, ck, cv, cdo
+
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
     if not args.no_e2e:
@@ -460,6 +501,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the separate FP8 forward measurement")
     ap.add_argument("--no-decode", action="store_true", help="skip the separate decode (split-KV) measurement")
+    ap.add_argument("--no-cp", action="store_true", help="skip the context-parallel (ring) measurement")
+    ap.add_argument("--cp-ranks", type=int, default=4, help="ranks of the context-parallel ring measurement")
     ap.add_argument("--decode-workload", default="decode70b", help="KV-history workload of the decode measurement")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -153,6 +153,42 @@ FA_API fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void
                                 const void* o, const void* dout, const float* lse,
                                 void* dq, void* dk, void* dv, void* stream);
 
+/* ---- Sequence-sharded (context-parallel) attention.
+ * "【词汇专栏】FlashAttention：大模型训练的加速器" (section 3.2, item 2) splits a
+ * long sequence across devices, each working on its part.  The exact join of
+ * the per-part results is the log-sum-exp merge below (adding the parts'
+ * outputs, as the page puts it, is not attention).  A device runs fa_fwd and
+ * fa_bwd on (query chunk, key chunk) pairs of equal length, with
+ * causal = 1 on the diagonal pair and 0 below it, and joins the results with
+ * these two kernels; the ring schedule and the exchange of K/V chunks between
+ * devices live in the Python package (context_parallel.py).  fa_bwd on a pair
+ * takes the FULL row statistics (the merged O and LSE of its query chunk), so
+ * each pair's dQ, dK, dV are exact terms of the whole-sequence gradient.
+ *
+ * fa_lse_merge merges a partial result over one block of keys into a running
+ * result over other keys.  rows = number of query rows (B*Hq*Nq), D in {64, 128}.
+ *   o_part   bf16 [rows, D]  result normalised over the block (as fa_fwd writes it)
+ *   lse_part fp32 [rows]     its natural-log LSE (-inf: the row saw no key of the block)
+ *   o_acc    fp32 [rows, D]  running result, normalised over the keys merged so far (in/out)
+ *   lse_acc  fp32 [rows]     its LSE (in/out)
+ *   o_out    bf16 [rows, D]  optional (NULL allowed): also receives the merged result
+ *   first    nonzero: o_acc / lse_acc are not read and are set from the part
+ * lse = log(exp(lse_acc) + exp(lse_part)); o_acc = exp(lse_acc - lse) o_acc +
+ * exp(lse_part - lse) o_part.  Rows without mass on either side become 0 and
+ * -inf.  Device pointers, 16-byte aligned (lse pointers 4-byte aligned); the
+ * caller owns all of them.  rows == 0 reads nothing and launches nothing (the
+ * pointers may then be NULL).  FA_ERR_INVALID_ARG for rows < 0, null or
+ * misaligned pointers; FA_ERR_UNSUPPORTED for other D. */
+FA_API fa_status fa_lse_merge(long long rows, int D, const void* o_part, const float* lse_part, float* o_acc,
+                              float* lse_acc, void* o_out, int first, void* stream);
+
+/* Gradient accumulation: acc = (first ? 0 : acc) + src, elementwise over n
+ * elements (src bf16, acc fp32; src NULL adds nothing), and out = bf16(acc)
+ * when out is not NULL.  n >= 0 and a multiple of 8; device pointers 16-byte
+ * aligned, owned by the caller; n == 0 reads nothing and launches nothing
+ * (the pointers may then be NULL).  FA_ERR_INVALID_ARG otherwise. */
+FA_API fa_status fa_accumulate(long long n, const void* src, float* acc, void* out, int first, void* stream);
+
 /* Synchronises `stream`, then reports and clears the device status word of
  * the current device: FA_ERR_TIMEOUT if any kernel gave up a bounded wait
  * since the last call, FA_ERR_CUDA if the stream reports an error, else FA_OK. */
@@ -173,11 +209,12 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
  * preprocess, 2 fused backward (dK, dV and dQ by fp32 reductions), 3 dQ
  * convert, 4 backward dK/dV kernel, 5 backward dQ kernel, 6 FP8 forward, 7 decode
- * (split kernel and combine together) (FA_PROFILE_KINDS;
+ * (split kernel and combine together), 8 log-sum-exp merge, 9 accumulation
+ * (FA_PROFILE_KINDS;
  * fa_bwd uses 1, 4, 5 by default and 1, 2, 3 when the environment variable
  * FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
  * objects; no device memory is allocated. */
-#define FA_PROFILE_KINDS 8
+#define FA_PROFILE_KINDS 10
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

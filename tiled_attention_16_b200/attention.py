@@ -74,6 +74,11 @@ def lib() -> ctypes.CDLL:
         L.fa_debug_timeout_sites.restype = ctypes.c_uint
         L.fa_bwd_noalloc.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.fa_bwd_noalloc.restype = ctypes.c_int
+        ll = ctypes.c_longlong
+        L.fa_lse_merge.argtypes = [ll, ctypes.c_int, vp, vp, vp, vp, vp, ctypes.c_int, vp]
+        L.fa_lse_merge.restype = ctypes.c_int
+        L.fa_accumulate.argtypes = [ll, vp, vp, vp, ctypes.c_int, vp]
+        L.fa_accumulate.restype = ctypes.c_int
         L.fa_profile_begin.argtypes = []
         L.fa_profile_begin.restype = ctypes.c_int
         L.fa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
@@ -271,6 +276,43 @@ def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None =
     return dq, dk, dv
 
 
+def lse_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, lse_part: torch.Tensor,
+              first: bool = False, out: torch.Tensor | None = None) -> None:
+    """Merge a partial result (o_part bf16 [..., D], lse_part fp32 [...]) over
+    one block of keys into the running result (o_acc fp32 [..., D], lse_acc
+    fp32 [...]) in place, by the log-sum-exp rule (fa_lse_merge).  With
+    first=True the running result is set from the part.  `out` (bf16, shaped
+    like o_part) also receives the merged result when given."""
+    D = o_part.shape[-1]
+    rows = o_part.numel() // D if D else 0
+    _check(o_part, "o_part", o_part.shape)
+    _check(o_acc, "o_acc", o_part.shape, torch.float32)
+    _check(lse_part, "lse_part", o_part.shape[:-1], torch.float32)
+    _check(lse_acc, "lse_acc", o_part.shape[:-1], torch.float32)
+    if out is not None:
+        _check(out, "out", o_part.shape)
+    st = lib().fa_lse_merge(rows, int(D), o_part.data_ptr(), lse_part.data_ptr(), o_acc.data_ptr(),
+                            lse_acc.data_ptr(), None if out is None else out.data_ptr(), 1 if first else 0,
+                            _stream_ptr(o_part.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_lse_merge")
+
+
+def accumulate(acc: torch.Tensor, src: torch.Tensor | None, first: bool = False,
+               out: torch.Tensor | None = None) -> None:
+    """acc (fp32) = (0 if first else acc) + src (bf16, same shape; None adds
+    nothing), in place (fa_accumulate); `out` (bf16) also receives bf16(acc)."""
+    _check(acc, "acc", acc.shape, torch.float32)
+    if src is not None:
+        _check(src, "src", acc.shape)
+    if out is not None:
+        _check(out, "out", acc.shape)
+    st = lib().fa_accumulate(acc.numel(), None if src is None else src.data_ptr(), acc.data_ptr(),
+                             None if out is None else out.data_ptr(), 1 if first else 0, _stream_ptr(acc.device))
+    if st != FA_OK:
+        raise FAError(st, "fa_accumulate")
+
+
 def device_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     dev = torch.device("cuda") if device is None else torch.device(device)
@@ -282,7 +324,8 @@ def timeout_sites() -> int:
 
 
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
-                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode")
+                 "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode",
+                 "fa_lse_merge_kernel", "fa_accumulate_kernel")
 
 
 def profile_begin() -> None:

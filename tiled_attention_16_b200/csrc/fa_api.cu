@@ -474,6 +474,36 @@ fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, co
     return fa_bwd(shape, q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+fa_status fa_lse_merge(long long rows, int D, const void* o_part, const float* lse_part, float* o_acc,
+                       float* lse_acc, void* o_out, int first, void* stream) {
+    if (rows < 0) return FA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+    if (rows == 0) return FA_OK;  // nothing is read; empty tensors may carry null pointers
+    if (!aligned16(o_part) || !aligned16(o_acc) || (o_out != nullptr && !aligned16(o_out))) return FA_ERR_INVALID_ARG;
+    if (lse_part == nullptr || lse_acc == nullptr || (reinterpret_cast<uintptr_t>(lse_part) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(lse_acc) & 3u) != 0)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_device();
+    if (st != FA_OK) return st;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed(8, strm, [&] {
+        return launch_lse_merge(D, rows, o_part, lse_part, o_acc, lse_acc, o_out, first, strm);
+    });
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_accumulate(long long n, const void* src, float* acc, void* out, int first, void* stream) {
+    if (n < 0 || (n & 7) != 0) return FA_ERR_INVALID_ARG;
+    if (n == 0) return FA_OK;  // nothing is read; empty tensors may carry null pointers
+    if (!aligned16(acc) || (src != nullptr && !aligned16(src)) || (out != nullptr && !aligned16(out)))
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_device();
+    if (st != FA_OK) return st;
+    cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    cudaError_t e = timed(9, strm, [&] { return launch_accumulate(n, src, acc, out, first, strm); });
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_get_device_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
     unsigned int word = 0;

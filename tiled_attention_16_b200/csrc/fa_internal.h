@@ -98,4 +98,10 @@ cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, c
 
 cudaError_t launch_bwd_dq_convert(const float* dq_acc, void* dq, size_t n_elems, cudaStream_t stream);
 
+// Sequence-sharded attention: log-sum-exp merge of a partial result into a
+// running one, and fp32 accumulation of bf16 gradient terms (fa_cp.cu).
+cudaError_t launch_lse_merge(int D, long long rows, const void* o_part, const float* lse_part, float* o_acc,
+                             float* lse_acc, void* o_out, int first, cudaStream_t stream);
+cudaError_t launch_accumulate(long long n, const void* src, float* acc, void* out, int first, cudaStream_t stream);
+
 }  // namespace fa
