@@ -242,7 +242,7 @@ def run_gpu(args, wl):
     import torch.distributed as dist
     from tiled_attention_16_b200 import attention as A
     from tiled_attention_16_b200.build import build
-    from tiled_attention_16_b200.workloads import make_inputs
+    from tiled_attention_16_b200.workloads import WORKLOADS, make_inputs
 
     ws, rank, local = dist_env()
     if ws > 1:
@@ -387,46 +387,64 @@ def run_gpu(args, wl):
             "peak_source": f"{peak_src} hbm_gbs", "launches": nd, "timed_alone": True}
         del dq_, dk_, dv_, dws, do_, dlse
 
-    # context parallel: the ring of CP_RANKS ranks over this workload's sequence
-    # (zigzag chunks), all ranks' pairs run on this one GPU in ring order; the
-    # exchange is not timed (it needs more GPUs).  Same flop convention as
-    # the step, so the ratio to the step's rate is the chunking's cost.
-    if not args.no_cp and wl.N % (2 * args.cp_ranks) == 0:
+    # context parallel: a ring of --cp-ranks ranks over a long sequence
+    # (--cp-workload, zigzag chunks), every rank's pairs run on this one GPU
+    # in ring order; the exchange is not timed (it needs more GPUs).  The
+    # single-kernel path is timed on the same inputs, so the ratio of the two
+    # rates is what chunking, merging and accumulating cost.
+    cwl = WORKLOADS[args.cp_workload]
+    if not args.no_cp and cwl.N % (2 * args.cp_ranks) == 0:
         from tiled_attention_16_b200 import context_parallel as cp
         R = args.cp_ranks
+        cq, ck, cv, cdo = (x.to(dev) for x in make_inputs(rank_workload(cwl, rank)))
         sh = lambda x: [cp.shard_sequence(x, r, R) for r in range(R)]  # noqa: E731
-        cq, ck, cv, cdo = sh(q), sh(k), sh(v), sh(do)
+        sq, sk, sv, sdo = sh(cq), sh(ck), sh(cv), sh(cdo)
 
         def ring_step():
-            fw = cp.virtual_ring_fwd(cq, ck, cv, wl.causal, wl.softmax_scale)
-            cp.virtual_ring_bwd(cq, ck, cv, [f[0] for f in fw], cdo, [f[1] for f in fw], wl.causal,
-                                wl.softmax_scale)
+            fw = cp.virtual_ring_fwd(sq, sk, sv, cwl.causal, cwl.softmax_scale)
+            cp.virtual_ring_bwd(sq, sk, sv, [f[0] for f in fw], sdo, [f[1] for f in fw], cwl.causal,
+                                cwl.softmax_scale)
 
-        for _ in range(3):
-            ring_step()
-        torch.cuda.synchronize()
-        A.profile_begin()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
+        cws = torch.empty(A.workspace_bytes(cwl.B, cwl.Hq, cwl.Hkv, cwl.N, cwl.D), device=dev, dtype=torch.uint8)
+
+        def mono_step():
+            co, clse = A.fwd(cq, ck, cv, causal=cwl.causal)
+            A.bwd(cq, ck, cv, co, cdo, clse, causal=cwl.causal, workspace=cws)
+
+        def timed_ms(fn, n):
+            for _ in range(3):
+                fn()
+            torch.cuda.synchronize()
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record()
+            for _ in range(n):
+                fn()
+            t1.record()
+            torch.cuda.synchronize()
+            return t0.elapsed_time(t1) / n
+
         n_cp = 5
-        for _ in range(n_cp):
-            ring_step()
-        e1.record()
-        torch.cuda.synchronize()
+        mono_ms = timed_ms(mono_step, n_cp)
+        A.profile_begin()
+        cp_ms = timed_ms(ring_step, n_cp)
         cp_kernels = A.profile_end()
         if A.device_status(dev) != A.FA_OK:
             raise RuntimeError("device status not OK after the context-parallel ring")
-        cp_ms = e0.elapsed_time(e1) / n_cp
-        cp_tf = flops_step / (cp_ms * 1e-3) / 1e12
-        step_tf = flops_step / (ms * 1e-3) / 1e12
+        cflops = cwl.flops_fwd() + cwl.flops_bwd()
+        cp_tf = cflops / (cp_ms * 1e-3) / 1e12
+        mono_tf = cflops / (mono_ms * 1e-3) / 1e12
+        n_all = n_cp + 3
         breakdown["context_parallel"] = {
-            "ranks": R, "chunk_rows": wl.N // (2 * R), "layout": "zigzag", "ms_per_step": cp_ms,
-            "tflops": cp_tf, "vs_step_rate": cp_tf / step_tf if step_tf else None,
-            "merge_ms": cp_kernels["fa_lse_merge_kernel"][0] / n_cp,
-            "accumulate_ms": cp_kernels["fa_accumulate_kernel"][0] / n_cp,
-            "launches_per_step": sum(nn for _, nn in cp_kernels.values()) / n_cp,
+            "workload": f"{cwl.name}: B={cwl.B} Hq={cwl.Hq} Hkv={cwl.Hkv} N={cwl.N} D={cwl.D}"
+                        f"{' causal' if cwl.causal else ''}",
+            "ranks": R, "chunk_rows": cwl.N // (2 * R), "layout": "zigzag",
+            "ms_per_step": cp_ms, "tflops": cp_tf, "single_kernel_ms": mono_ms, "single_kernel_tflops": mono_tf,
+            "vs_single_kernel": cp_tf / mono_tf,
+            "merge_ms": cp_kernels["fa_lse_merge_kernel"][0] / n_all,
+            "accumulate_ms": cp_kernels["fa_accumulate_kernel"][0] / n_all,
+            "launches_per_step": sum(nn for _, nn in cp_kernels.values()) / n_all,
             "exchange": "not timed (one GPU): the ranks run one after another on it", "timed_alone": True}
-        del cq, ck, cv, cdo
+        del cq, ck, cv, cdo, sq, sk, sv, sdo, cws
 
     # end to end through the public API with host buffers (pinned), copies timed
     e2e = None
@@ -503,6 +521,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the separate decode (split-KV) measurement")
     ap.add_argument("--no-cp", action="store_true", help="skip the context-parallel (ring) measurement")
     ap.add_argument("--cp-ranks", type=int, default=4, help="ranks of the context-parallel ring measurement")
+    ap.add_argument("--cp-workload", default="stress", help="sequence of the context-parallel ring measurement")
     ap.add_argument("--decode-workload", default="decode70b", help="KV-history workload of the decode measurement")
     args = ap.parse_args()
     if args.warmup < 3:
