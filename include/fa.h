@@ -113,8 +113,11 @@ FA_API fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* 
                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for `shape` (0 if the shape is invalid):
- * the per-row statistics (LSE in log2 units and D = rowsum(dO o O), each
- * padded to a multiple of 128 rows) and an fp32 dQ accumulator [B,Hq,N,D]. */
+ * two work counters and the per-row statistics (LSE in log2 units and
+ * D = rowsum(dO o O), each padded to a multiple of 128 rows), about
+ * 8 * B * Hq * N bytes; plus an fp32 dQ accumulator [B,Hq,N,D] when the
+ * environment variable FA_DQ_MODE=atomic selects the fused backward (the
+ * mode is read once per process, so the size is stable within a process). */
 FA_API size_t fa_bwd_workspace_bytes(const fa_shape* shape);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16) and lse (fp32, as written by
@@ -131,7 +134,7 @@ FA_API fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, con
  *
  * Same computation, arguments and outputs as fa_bwd, but without a caller
  * workspace: the scratch it needs (the per-row LSE/D statistics and the fp32
- * dQ accumulator, fa_bwd_workspace_bytes(shape) bytes) lives in a fixed
+ * dQ accumulator of the fused mode, fa_bwd_workspace_bytes(shape) bytes) lives in a fixed
  * FA_NOALLOC_SCRATCH_BYTES region of device memory that the library reserves
  * statically on every GPU that loads it, held until the process exits.  It is
  * meant for callers that cannot call cudaMalloc or hand out device memory on

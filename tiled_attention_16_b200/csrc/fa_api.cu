@@ -379,7 +379,7 @@ fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* k, cons
 
 size_t fa_bwd_workspace_bytes(const fa_shape* shape) {
     if (check_shape(shape) != FA_OK) return 0;
-    return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D).total;
+    return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total;
 }
 
 fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -391,7 +391,8 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
     const fa_shape& s = *shape;
-    const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D);
+    const bool separate = dq_separate_mode();
+    const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D, !separate);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws.total)
         return FA_ERR_INVALID_ARG;
     if ((st = check_device()) != FA_OK) return st;
@@ -408,7 +409,6 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.N = s.N;
     p.Npad = Npad;
     p.causal = s.causal ? 1 : 0;
-    const bool separate = dq_separate_mode();
     const int T = (s.N + kTileM - 1) / kTileM;
     // K/V heads per scheduling group of the key-block kernels: keep the
     // group's Q, dO (bf16) and, for the fused kernel, the fp32 dQ accumulator
@@ -430,7 +430,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
     p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2_off);
     p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec_off);
-    p.dq_acc = reinterpret_cast<float*>(wsb + ws.dq_off);
+    p.dq_acc = separate ? nullptr : reinterpret_cast<float*>(wsb + ws.dq_off);
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
@@ -466,7 +466,8 @@ fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, co
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
-    if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D).total > FA_NOALLOC_SCRATCH_BYTES)
+    if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total >
+        FA_NOALLOC_SCRATCH_BYTES)
         return FA_ERR_TOO_LARGE;
     if ((st = check_device()) != FA_OK) return st;
     void* scratch = nullptr;

@@ -570,7 +570,7 @@ int grid_for(size_t work, int per_block) {
 
 }  // namespace
 
-BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D) {
+BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D, bool with_dq_acc) {
     auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
     const size_t BH = static_cast<size_t>(B) * Hq;
     const size_t Npad = (static_cast<size_t>(N) + kTileM - 1) / kTileM * kTileM;
@@ -579,7 +579,7 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D) {
     w.lse2_off = up(kSchedCounters * 4);
     w.dvec_off = w.lse2_off + up(BH * Npad * 4);
     w.dq_off = w.dvec_off + up(BH * Npad * 4);
-    w.total = w.dq_off + up(BH * static_cast<size_t>(N) * D * 4);
+    w.total = w.dq_off + (with_dq_acc ? up(BH * static_cast<size_t>(N) * D * 4) : 0);
     return w;
 }
 

@@ -70,7 +70,9 @@ cudaError_t launch_decode(int D, const CUtensorMap& tk, const CUtensorMap& tv, c
 struct BwdWorkspace {
     size_t sched_off, lse2_off, dvec_off, dq_off, total;
 };
-BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D);
+// with_dq_acc: room for the fp32 dQ accumulator of the fused kernel (dq_off ..
+// total); the default separate dQ pass needs none (dq_off == total).
+BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D, bool with_dq_acc);
 
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, cudaStream_t stream);
