@@ -45,6 +45,7 @@ constexpr int kLoadWarp = kComputeWarps + 1;
 constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr int kCompute = 32 * kComputeWarps;
 static_assert(kCols % 32 == 0, "each compute thread handles whole 32-column TMEM loads");
+static_assert(kCols == 64, "the dK/dV pass hands P^T to the dV MMAs in two 32-column halves per group");
 constexpr int kMaxDynSmem = 232448;
 
 // wait sites (bits of the device status word)
@@ -84,7 +85,7 @@ struct DkdvLayout {
     static constexpr int kLse = kDO + 2 * kTileBytes;
     static constexpr int kDvec = kLse + 2 * kTileN * 4;
     static constexpr int kBar = kDvec + 2 * kTileN * 4;
-    static constexpr int kNumBars = 20;
+    static constexpr int kNumBars = 21;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -165,13 +166,14 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint64_t* do_empty = bars + 7;     // [2]
     uint64_t* s_full = bars + 9;
     uint64_t* dp_full = bars + 10;
-    uint64_t* p_full = bars + 11;
+    uint64_t* p_full0 = bars + 11;     // P^T of each group's first 32 query columns
     uint64_t* ds_full = bars + 12;
     uint64_t* dkv_full = bars + 13;
     uint64_t* drain = bars + 14;
     uint64_t* kv_empty = bars + 15;
     uint64_t* unit_full = bars + 16;   // [2]
     uint64_t* unit_empty = bars + 18;  // [2]
+    uint64_t* p_full1 = bars + 20;     // P^T of each group's last 32 query columns
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
@@ -195,7 +197,8 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
         mbar_init(s_full, 1);
         mbar_init(dp_full, 1);
-        mbar_init(p_full, kCompute);
+        mbar_init(p_full0, kCompute);
+        mbar_init(p_full1, kCompute);
         mbar_init(ds_full, kCompute);
         mbar_init(dkv_full, 1);
         mbar_init(drain, 1);
@@ -338,13 +341,24 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     }
                     tc_commit(dp_full);
                     if (it == n_it - 1) tc_commit(kv_empty);   // K and V no longer read by this unit
-                    // dV += P^T dO
-                    if (!(ok = mbar_wait(p_full, ph, abort_flag, kS1Mma))) break;
-                    tc_fence_after();
+                    // dV += P^T dO, in two halves of every group's query columns:
+                    // the first half's MMAs run while the compute warps still
+                    // form the second half of P^T
 #pragma unroll
-                    for (int kk = 0; kk < kTileM / 16; ++kk)
-                        mma_ts(tmem + kColDV, tmem + kColS + packed_col(kk), sdesc_sw128(da + kk * 2048, kAtom, 1024),
-                               kIdAcc, (it > 0 || kk > 0));
+                    for (int h = 0; h < 2; ++h) {
+                        if (!(ok = mbar_wait(h == 0 ? p_full0 : p_full1, ph, abort_flag, kS1Mma))) break;
+                        tc_fence_after();
+#pragma unroll
+                        for (int g2 = 0; g2 < kGroups; ++g2) {
+#pragma unroll
+                            for (int t = 0; t < kCols / 32; ++t) {
+                                const int kk = g2 * (kCols / 16) + h * (kCols / 32) + t;
+                                mma_ts(tmem + kColDV, tmem + kColS + packed_col(kk),
+                                       sdesc_sw128(da + kk * 2048, kAtom, 1024), kIdAcc, (it > 0 || kk > 0));
+                            }
+                        }
+                    }
+                    if (!ok) break;
                     tc_commit(&do_empty[st]);
                 }
                 if (!ok) break;
@@ -400,30 +414,33 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                     // last key block (both uniform across the warp); there,
                     // columns q < lo are zero (lo = kCols masks a key row past N).
                     const bool diag = p.causal && (i == j);
+                    const bool masked = diag || kv_block_partial;
+                    const int lo = !kv_ok ? kCols : (diag ? r - c0 : 0);
                     const float2 c2 = make_float2(c, c);
-                    static_for<0, kCols / 2>([&](auto tc) {
-                        constexpr int q = 2 * decltype(tc)::value;
-                        const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
-                        const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
-                        pv[q] = exp2_mixed<q>(x.x);
-                        pv[q + 1] = exp2_mixed<q + 1>(x.y);
-                    });
-                    if (diag || kv_block_partial) {
-                        const int lo = !kv_ok ? kCols : (diag ? r - c0 : 0);
+                    // two halves of 32 columns, each handed to the dV MMAs as
+                    // soon as it is in TMEM (p_full0, p_full1)
+                    static_for<0, 2>([&](auto hh) {
+                        constexpr int h = decltype(hh)::value;
+                        static_for<0, 16>([&](auto tc) {
+                            constexpr int q = 32 * h + 2 * decltype(tc)::value;
+                            const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
+                            const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
+                            pv[q] = exp2_mixed<q>(x.x);
+                            pv[q + 1] = exp2_mixed<q + 1>(x.y);
+                        });
+                        if (masked) {
 #pragma unroll
-                        for (int q = 0; q < kCols; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
-                    }
-#pragma unroll
-                    for (int h = 0; h < kCols / 32; ++h) {
+                            for (int q = 32 * h; q < 32 * h + 32; ++q) pv[q] = (q >= lo) ? pv[q] : 0.f;
+                        }
                         uint32_t pk[16];
 #pragma unroll
                         for (int t = 0; t < 16; ++t) pk[t] = pack_bf16x2(pv[32 * h + 2 * t], pv[32 * h + 2 * t + 1]);
                         tmem_st16(tmem + lane_off + kColS + c0 + h * 16, pk);
-                    }
-                    tmem_st_wait();
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(h == 0 ? p_full0 : p_full1);
+                    });
                 }
-                tc_fence_before();
-                mbar_arrive(p_full);
                 ok = mbar_wait(dp_full, ph, abort_flag, kS1Compute);
                 if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
                 tc_fence_after();
@@ -481,7 +498,7 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 }
             }
             // the next unit's dV / dK MMAs overwrite these columns only after this
-            // group's next P^T arrival (p_full), which follows these completed loads
+            // group's next P^T arrival (p_full0), which follows these completed loads
             tc_fence_before();
             g += w.n_it;
         }

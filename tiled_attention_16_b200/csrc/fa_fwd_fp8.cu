@@ -46,7 +46,7 @@ struct F8Layout {
     static constexpr int kK = kQ + 2 * kTileBytes;     // kF8Stages tiles
     static constexpr int kV = kK + kF8Stages * kTileBytes;
     static constexpr int kBar = kV + kF8Stages * kTileBytes;
-    static constexpr int kNumBars = 1 + 3 * kF8Stages + 3 * 2 + 1 + 1 + 2 * 2;  // ... drain, q_empty, unit ring
+    static constexpr int kNumBars = 1 + 3 * kF8Stages + 3 * 2 + 1 + 1 + 2 * 2 + 2;  // ... unit ring, p_half0
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -182,6 +182,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
     uint64_t* q_empty = drain + 1;
     uint64_t* unit_full = q_empty + 1;           // [2]
     uint64_t* unit_empty = unit_full + 2;        // [2]
+    uint64_t* p_half0 = unit_empty + 2;          // [2] keys 0-63 of P in TMEM (p_full: all of P)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
@@ -201,6 +202,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         for (int s = 0; s < 2; ++s) {
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], kTileM);
+            mbar_init(&p_half0[s], kTileM);
             mbar_init(&o_full[s], 1);
             mbar_init(&unit_full[s], 1);
             mbar_init(&unit_empty[s], 2 * kTileM + 1);
@@ -288,13 +290,26 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 for (int kk = 0; kk < kF8D / 32; ++kk)  // 32 e4m3 = 32 bytes per K step
                     mma_f8_ss(tmem + s * 128, qd + ((kk * 32) >> 4), kd + ((kk * 32) >> 4), kIdS, kk > 0 ? 1u : 0u);
             };
-            auto issue_pv = [&](int s, int st, int j) {
+            // O += P V_j for keys 64h .. 64h+63 of the tile (P as e4m3 in TMEM)
+            auto issue_pv_half = [&](int s, int st, int j, int h) {
                 const uint64_t vd = v_desc + ((st * L::kTileBytes) >> 4);
                 const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
-                for (int kk = 0; kk < kTileN / 32; ++kk)  // 32 keys = 8 packed columns = 32 V rows
+                for (int t = 0; t < kTileN / 64; ++t) {  // 32 keys = 8 packed columns = 32 V rows
+                    const int kk = h * (kTileN / 64) + t;
                     mma_f8_ts(tmem + 256 + s * 128, tmem + s * 128 + kk * 8, vd + ((kk * 32 * 128) >> 4), kIdPV,
                               kk > 0 ? 1u : acc0);
+                }
+            };
+            // the first half's MMAs run while the softmax warps still form the second
+            auto issue_pv = [&](int s, int st, int j, uint32_t parity) -> bool {
+                if (!mbar_wait(&p_half0[s], parity, abort_flag, kF8P)) return false;
+                tc_fence_after();
+                issue_pv_half(s, st, j, 0);
+                if (!mbar_wait(&p_full[s], parity, abort_flag, kF8P)) return false;
+                tc_fence_after();
+                issue_pv_half(s, st, j, 1);
+                return true;
             };
             bool ok = true;
             int gk = 0;                // K/V tiles consumed (all units)
@@ -323,9 +338,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     const uint32_t sn_ph = ((G + 1) / kF8Stages) & 1;
                     if (!(ok = mbar_wait(&v_full[st], ph, abort_flag, kF8V))) break;
                     if (j < nkv[0]) {
-                        if (!(ok = mbar_wait(&p_full[0], (c0 + j) & 1, abort_flag, kF8P))) break;
-                        tc_fence_after();
-                        issue_pv(0, st, j);
+                        if (!(ok = issue_pv(0, st, j, (c0 + j) & 1))) break;
                         if (j == nkv[0] - 1) tc_commit(&o_full[0]);
                         if (j + 1 < nkv[0]) {
                             if (!(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
@@ -335,9 +348,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         }
                     }
                     if (j < nkv[1]) {
-                        if (!(ok = mbar_wait(&p_full[1], (c1 + j) & 1, abort_flag, kF8P))) break;
-                        tc_fence_after();
-                        issue_pv(1, st, j);
+                        if (!(ok = issue_pv(1, st, j, (c1 + j) & 1))) break;
                         if (j == nkv[1] - 1) tc_commit(&o_full[1]);
                     }
                     tc_commit(&kv_empty[st]);
@@ -419,6 +430,9 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 const float2 c2 = make_float2(c, c);
                 const float2 nm2 = make_float2(-msub, -msub);
                 float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                // O must be rescaled before any PV MMA of this tile starts: a warp
+                // that rescales hands over the first half of P only afterwards
+                const bool late = rescale && j > 0;
 #pragma unroll
                 for (int half = 0; half < 2; ++half) {
                     uint32_t pk[16];
@@ -433,12 +447,17 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                         pk[t] = pack_e4m3x4(p0, p1, p2, p3);
                     });
                     tmem_st16(tS + half * 16, pk);
+                    if (half == 0 && !late) {   // keys 0-63 of P to the PV MMAs now
+                        tmem_st_wait();
+                        tc_fence_before();
+                        mbar_arrive(&p_half0[s]);
+                    }
                 }
                 l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
                 // O <- alpha O (PV of the previous tile has completed: it was
                 // committed before this tile's S); done after P so the S row is
                 // no longer live in registers
-                if (rescale && j > 0) {
+                if (late) {
 #pragma unroll 1
                     for (int q = 0; q < kF8D / 32; ++q) {
                         uint32_t orow[32];
@@ -451,6 +470,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 }
                 tmem_st_wait();
                 tc_fence_before();
+                if (late) mbar_arrive(&p_half0[s]);
                 mbar_arrive(&p_full[s]);
             }
             if (!ok) break;
