@@ -330,6 +330,8 @@ def run_gpu(args, wl):
     roofline = {"kernel": dominant, "bound": "tensor", "achieved": achieved, "peak": peak_tf,
                 "unit": "TFLOP/s", "frac": achieved / peak_tf, "traffic": recorded_traffic(dominant, wl.name),
                 "peak_source": f"{peak_src} bf16_tflops (burst)", "per_launch_ms": tensor_k[dominant],
+                "frac_of_sustained_peak": (achieved / peaks["bf16_tflops_sustained"]
+                                           if peaks.get("bf16_tflops_sustained") else None),
                 "flops_per_launch": kernel_flops[dominant]}
     fwd_tf = wl.flops_fwd() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = wl.flops_bwd() / (bwd_ms * 1e-3) / 1e12
