@@ -34,9 +34,12 @@ reads K/V head h // (Hq // Hkv) (contiguous groups).  Causal means key j is
 visible to query i iff j <= i (for Nq new queries over an Nk-long K/V
 history, attention_forward_kv: iff j <= Nk - Nq + i).  lse is the natural log
 of the scaled logits.
-Parity status: every function here is pinned by tests/test_oracle_pins.py
+Parity status: every function here is pinned, by tests/test_oracle_pins.py
 (closed forms, invariants, hand-worked golden values, brute force, central
-finite differences and a torch autograd cross-check).
+finite differences and a torch autograd cross-check) and, for the
+sequence-sharded pieces at the end, tests/test_oracle_sequence_shards.py
+(a hand-worked merge, scalar brute force, key and query partitions against
+the full-sequence functions above, and a planted mistake).
 """
 from __future__ import annotations
 
