@@ -5,8 +5,8 @@ kernels (tests/cp_reference_ops.py).
 * every (query chunk, key chunk) pair at or below the diagonal is computed
   exactly once over all ranks and steps, the diagonal ones causally; causal
   work is equal on every rank;
-* the ring run in one process (virtual ranks) and over gloo with two and
-  three processes reproduces the full-sequence oracle's O, LSE, dQ, dK, dV.
+* the ring run in one process (virtual ranks) and over gloo with two, three
+  and four processes reproduces the full-sequence oracle's O, LSE, dQ, dK, dV.
 """
 import os
 import socket
@@ -133,7 +133,7 @@ def _ring_worker(rank, world, port, causal, out_q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (2, False)])
+@pytest.mark.parametrize("world,causal", [(2, True), (3, True), (4, True), (2, False)])
 def test_gloo_ring_matches_full_sequence(world, causal):
     port = _free_port()
     ctx = mp.get_context("spawn")
