@@ -197,6 +197,18 @@ FA_API fa_status fa_accumulate(long long n, const void* src, float* acc, void* o
  * since the last call, FA_ERR_CUDA if the stream reports an error, else FA_OK. */
 FA_API fa_status fa_get_device_status(void* stream);
 
+/* Self-test of the failure detection (computes no attention).  Launches on
+ * `stream` one CTA whose thread waits, with the bounded wait every kernel of
+ * the library uses, on a barrier that nothing completes; at the wait limit
+ * (2 s) it records `site` in the device status word and raises the CTA's
+ * abort flag.  A second thread of the CTA waits on another such barrier from
+ * a quarter of the limit later and must leave through the abort flag without
+ * recording `site2`.  Afterwards fa_get_device_status() reports
+ * FA_ERR_TIMEOUT and fa_debug_timeout_sites() returns bit `site` alone; the
+ * CUDA context stays usable.  site and site2 in 0..31 and distinct, else
+ * FA_ERR_INVALID_ARG before any launch; FA_ERR_CUDA if the launch fails. */
+FA_API fa_status fa_selftest_wait_timeout(int site, int site2, void* stream);
+
 /* Static description of a status code. */
 FA_API const char* fa_status_str(fa_status status);
 

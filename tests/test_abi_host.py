@@ -21,7 +21,7 @@ def test_exports_every_declared_symbol():
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
                           "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
                           "fa_bwd_noalloc", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes",
-                          "fa_lse_merge", "fa_accumulate"}
+                          "fa_lse_merge", "fa_accumulate", "fa_selftest_wait_timeout"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -254,3 +254,8 @@ def test_merge_and_accumulate_valid_calls_fail_cleanly_without_gpu():
     # argument checks and stops at the device check
     assert _merge(lse_acc=P + 4) in (A.FA_ERR_CUDA, A.FA_ERR_UNSUPPORTED)
     assert _acc() in (A.FA_ERR_CUDA, A.FA_ERR_UNSUPPORTED)
+
+
+def test_selftest_rejects_bad_sites_before_launch():
+    for a, b in ((-1, 0), (0, 32), (5, 5), (40, 1)):
+        assert A.lib().fa_selftest_wait_timeout(a, b, None) == A.FA_ERR_INVALID_ARG

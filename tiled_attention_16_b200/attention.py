@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.fa_lse_merge.restype = ctypes.c_int
         L.fa_accumulate.argtypes = [ll, vp, vp, vp, ctypes.c_int, vp]
         L.fa_accumulate.restype = ctypes.c_int
+        L.fa_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_int, vp]
+        L.fa_selftest_wait_timeout.restype = ctypes.c_int
         L.fa_profile_begin.argtypes = []
         L.fa_profile_begin.restype = ctypes.c_int
         L.fa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
@@ -317,6 +319,15 @@ def device_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     dev = torch.device("cuda") if device is None else torch.device(device)
     return int(lib().fa_get_device_status(_stream_ptr(dev)))
+
+
+def selftest_wait_timeout(site: int, site2: int, device=None) -> None:
+    """Launch the failure-detection self-test (fa_selftest_wait_timeout) on the
+    current stream; read the outcome with device_status() and timeout_sites()."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    st = lib().fa_selftest_wait_timeout(int(site), int(site2), _stream_ptr(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_selftest_wait_timeout")
 
 
 def timeout_sites() -> int:
