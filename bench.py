@@ -113,6 +113,7 @@ class ClockSampler:
 COMMON_SOURCES = ("fa_api.cu", "sm100.cuh", "fa_internal.h")
 KERNEL_FILES = {
     "fa_fwd_kernel": ("fa_fwd.cu",),
+    "fa_fwd_pair_kernel": ("fa_fwd_pair.cu",),
     "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu",),
     "fa_bwd_dkdv_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
@@ -120,7 +121,7 @@ KERNEL_FILES = {
     "fa_decode_split_kernel": ("fa_decode.cu",),
     "fa_decode_combine_kernel": ("fa_decode.cu",),
 }
-TRAFFIC_GLOB = os.path.join(ROOT, "profiles", "dram_traffic_*.md")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "dram_traffic.json")
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -133,21 +134,18 @@ def kernel_source_hash(kernel: str) -> str:
 
 
 def recorded_traffic(kernel: str, workload: str):
-    """DRAM bytes (read + write) per launch from the committed ncu summaries
-    (profiles/dram_traffic_*.md), or None when there is none for this kernel
-    and workload or it was taken on other kernel sources.  The summaries'
-    table rows read `| kernel | workload | source hash | read bytes | write bytes | ... |`."""
-    import glob
+    """DRAM bytes (read + write) per launch from the committed ncu record
+    (profiles/dram_traffic.json), or None when there is none for this kernel
+    and workload or it was taken on other kernel sources."""
+    try:
+        with open(TRAFFIC_RECORD) as f:
+            entries = json.load(f)["entries"]
+    except (OSError, ValueError, KeyError):
+        return None
     src = kernel_source_hash(kernel)
-    for path in sorted(glob.glob(TRAFFIC_GLOB)):
-        with open(path) as f:
-            for line in f:
-                cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
-                if len(cells) >= 5 and cells[0] == kernel and cells[1] == workload and cells[2] == src:
-                    try:
-                        return int(cells[3]) + int(cells[4])
-                    except ValueError:
-                        return None
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload and e.get("source_hash") == src:
+            return int(e["read_bytes"]) + int(e["write_bytes"])
     return None
 
 
@@ -314,15 +312,17 @@ def run_gpu(args, wl):
 
     # kernel-level numbers from the live events
     kms = {k: (t / n if n else None) for k, (t, n) in per_kernel.items()}
-    fwd_ms = kms["fa_fwd_kernel"]
-    bwd_ms = sum(x for k, x in kms.items() if k != "fa_fwd_kernel" and x)
+    fwd_kinds = ("fa_fwd_kernel", "fa_fwd_pair_kernel")
+    fwd_kernel = max(fwd_kinds, key=lambda k: kms[k] or 0.0)   # the forward kernel the step ran
+    fwd_ms = kms[fwd_kernel]
+    bwd_ms = sum(x for k, x in kms.items() if k not in fwd_kinds and x)
     peaks, peak_src = load_peaks()
     peak_tf = peaks["bf16_tflops"]
     # GEMM flops each tensor kernel executes (one "GEMM" over a head = 2*N^2*D,
     # halved when causal): fused backward 5, dK/dV kernel 4 (S, dP, dV, dK),
     # dQ kernel 3 (S and dP recomputed, dQ).
     gemm = wl.flops_fwd() / 2
-    kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
+    kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_fwd_pair_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
                     "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm}
     tensor_k = {k: v for k, v in kms.items() if v and k in kernel_flops}
     dominant = max(tensor_k, key=lambda k: tensor_k[k])
@@ -342,7 +342,8 @@ def run_gpu(args, wl):
         "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_of_peak": fwd_tf / peak_tf,
         "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_of_peak": bwd_tf / peak_tf,
         "bwd_mode": "separate dQ pass" if kms.get("fa_bwd_dq_kernel") else "fused (fp32 dQ reductions)",
-        "bwd_kernels_ms": {k: v for k, v in kms.items() if v and k != "fa_fwd_kernel"},
+        "fwd_kernel": fwd_kernel,
+        "bwd_kernels_ms": {k: v for k, v in kms.items() if v and k not in fwd_kinds},
         "bwd_preprocess_gbs": pre_bytes / (kms["fa_bwd_preprocess"] * 1e-3) / 1e9 if kms["fa_bwd_preprocess"] else None,
         "bwd_dq_convert_gbs": conv_bytes / (kms["fa_bwd_dq_convert"] * 1e-3) / 1e9 if kms["fa_bwd_dq_convert"] else None,
         "hbm_peak_gbs": peaks["hbm_gbs"],

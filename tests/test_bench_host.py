@@ -7,6 +7,7 @@
 * the throughput arithmetic of the JSON line.
 """
 import datetime
+import json
 import os
 import sys
 import time
@@ -67,27 +68,27 @@ def test_traffic_record_follows_the_source_hash(tmp_path, monkeypatch):
     k = "fa_fwd_kernel"
     h = bench.kernel_source_hash(k)
     assert len(h) == 16 and h == bench.kernel_source_hash(k)
-    summary = tmp_path / "dram_traffic_x.md"
-    summary.write_text("| kernel | workload | source hash | read bytes | write bytes | ns |\n|---|---|---|---|---|---|\n"
-                       f"| {k} | wl | {h} | 100 | 23 | 5 |\n| {k} | wl2 | 0000000000000000 | 1 | 1 | 1 |\n")
-    monkeypatch.setattr(bench, "TRAFFIC_GLOB", str(tmp_path / "dram_traffic_*.md"))
+    rec = tmp_path / "dram_traffic.json"
+    rec.write_text(json.dumps({"entries": [
+        {"kernel": k, "workload": "wl", "source_hash": h, "read_bytes": 100, "write_bytes": 23},
+        {"kernel": k, "workload": "wl2", "source_hash": "0000000000000000", "read_bytes": 1, "write_bytes": 1}]}))
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(rec))
     assert bench.recorded_traffic(k, "wl") == 123
     assert bench.recorded_traffic(k, "wl2") is None        # taken on other sources
     assert bench.recorded_traffic(k, "other") is None
     assert bench.recorded_traffic("fa_bwd_dq_kernel", "wl") is None
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", str(tmp_path / "missing.json"))
+    assert bench.recorded_traffic(k, "wl") is None
 
 
-def test_committed_traffic_records_parse():
-    # every row of the committed summaries names a known kernel and integer byte counts
-    import glob
-    rows = 0
-    for path in glob.glob(os.path.join(ROOT, "profiles", "dram_traffic_*.md")):
-        for line in open(path):
-            cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 6 and cells[0] in bench.KERNEL_FILES and len(cells[2]) == 16:
-                int(cells[3]), int(cells[4])
-                rows += 1
-    assert rows >= 6
+def test_committed_traffic_record_parses():
+    # every entry of the committed record names a known kernel and integer byte counts
+    with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+        entries = json.load(f)["entries"]
+    for e in entries:
+        assert e["kernel"] in bench.KERNEL_FILES and len(e["source_hash"]) == 16
+        int(e["read_bytes"]), int(e["write_bytes"])
+    assert len(entries) >= 6
 
 
 @pytest.mark.parametrize("ws", [1, 2, 8])
