@@ -29,7 +29,19 @@
  *
  * Ownership.  The caller allocates and owns every buffer (device memory),
  * including the backward workspace.  The library allocates no device memory on
- * these calls.  Pointers must be device pointers aligned to 16 bytes.
+ * these calls.  Pointers must be device pointers aligned to 16 bytes (the
+ * backward's lse input: 4 bytes, it is read one element at a time).
+ *
+ * Streams and CUDA graphs.  The persistent forward kernels (fa_fwd,
+ * fa_fwd_fp8) hand out work through a counter in a small static device table
+ * of the library.  A launch outside stream capture takes one of 1024 slots in
+ * turn, so launches that overlap on different streams use different counters;
+ * a launch recorded into a CUDA graph takes a slot reserved for captured
+ * launches (3072 of them, in turn), which no eager launch ever uses.  Two
+ * replays of the same graph that run at the same time share that graph's
+ * counters, like every other buffer the graph names, and must not overlap.
+ * The first call on a device looks up the table's address, so make it before
+ * capturing on that device.
  *
  * Asynchrony and errors.  Calls enqueue kernels on `stream` and return at
  * once.  A non-OK status means nothing was launched (argument errors) or the
@@ -121,7 +133,7 @@ FA_API fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* 
 FA_API size_t fa_bwd_workspace_bytes(const fa_shape* shape);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16) and lse (fp32, as written by
- * fa_fwd).  Outputs dq [B,Hq,N,D], dk and dv [B,Hkv,N,D], bf16, overwritten.
+ * fa_fwd; 4-byte alignment suffices).  Outputs dq [B,Hq,N,D], dk and dv [B,Hkv,N,D], bf16, overwritten.
  * `workspace` must be a device buffer of at least fa_bwd_workspace_bytes(shape)
  * bytes, 256-byte aligned; its contents on entry do not matter. */
 FA_API fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v,
@@ -221,15 +233,17 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * the library launches is bracketed by a pair of CUDA events recorded on the
  * launching stream.  fa_profile_end() waits for those events, writes for each
  * kernel kind k the summed duration total_ms[k] and the launch count
- * launches[k], and stops recording.  Kinds: 0 forward, 1 backward
- * preprocess, 2 fused backward (dK, dV and dQ by fp32 reductions), 3 dQ
- * convert, 4 backward dK/dV kernel, 5 backward dQ kernel, 6 FP8 forward, 7 decode
- * (split kernel and combine together), 8 log-sum-exp merge, 9 accumulation
- * (FA_PROFILE_KINDS;
+ * launches[k], and stops recording.  Kinds: 0 forward (one-CTA kernel,
+ * 128-row MMA tiles), 1 backward preprocess, 2 fused backward (dK, dV and dQ
+ * by fp32 reductions), 3 dQ convert, 4 backward dK/dV kernel, 5 backward dQ
+ * kernel, 6 FP8 forward, 7 decode (split kernel and combine together),
+ * 8 log-sum-exp merge, 9 accumulation, 10 forward on CTA pairs (256-row MMA
+ * tiles) (FA_PROFILE_KINDS; fa_fwd uses 0, or 10 when the environment
+ * variable FA_FWD_TILE=m256 selects the CTA-pair kernel for D = 128;
  * fa_bwd uses 1, 4, 5 by default and 1, 2, 3 when the environment variable
  * FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
  * objects; no device memory is allocated. */
-#define FA_PROFILE_KINDS 10
+#define FA_PROFILE_KINDS 11
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

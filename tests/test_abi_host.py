@@ -88,9 +88,19 @@ def test_fwd_bad_pointers(bad, which):
 
 
 @pytest.mark.parametrize("bad", [0, P + 4])
-@pytest.mark.parametrize("which", ["q", "k", "v", "o", "do", "lse", "dq", "dk", "dv"])
+@pytest.mark.parametrize("which", ["q", "k", "v", "o", "do", "dq", "dk", "dv"])
 def test_bwd_bad_pointers(bad, which):
     assert _bwd(shape(), **{which: bad}) == A.FA_ERR_INVALID_ARG
+
+
+def test_bwd_lse_alignment():
+    # the backward reads LSE one float at a time: 4-byte alignment is enough
+    assert _bwd(shape(), lse=0) == A.FA_ERR_INVALID_ARG
+    assert _bwd(shape(), lse=P + 2) == A.FA_ERR_INVALID_ARG
+    assert _noalloc(shape(), lse=P + 2) == A.FA_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():   # with a GPU this valid call would launch on the fake pointers
+        assert _bwd(shape(), lse=P + 4) in (A.FA_ERR_CUDA, A.FA_ERR_UNSUPPORTED)
 
 
 def test_bwd_workspace_checks():
@@ -131,7 +141,7 @@ def test_profile_hooks_without_launches():
     A.profile_begin()
     res = A.profile_end()
     assert set(res) == set(A.PROFILE_KINDS)
-    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 10
+    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 11
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
 
 

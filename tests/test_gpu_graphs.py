@@ -98,3 +98,54 @@ def test_decode_replays_bitwise():
     torch.cuda.synchronize()
     assert A.device_status(dev) == A.FA_OK
     assert torch.equal(o, ref_o) and torch.equal(lse, ref_l)
+
+
+def test_captured_forward_keeps_its_counter_slot():
+    """A forward recorded into a CUDA graph takes a work-counter slot that no
+    eager forward ever uses.  After more eager launches than the eager slot
+    ring holds (so every eager slot has been reused), graph replays that run
+    next to eager forwards on another stream still write every row, and both
+    match their eager results bit for bit."""
+    dev = _gpu()
+    wl = Workload("graph_slot", B=2, Hq=8, Hkv=8, N=2048, D=128, causal=True, seed=31)
+    q, k, v, _ = (x.to(dev) for x in make_inputs(wl))
+    o_g = torch.empty_like(q)
+    l_g = torch.empty(2, 8, 2048, device=dev, dtype=torch.float32)
+    A.fwd(q, k, v, causal=True, out=o_g, lse=l_g)   # eager first: one-time lookups outside capture
+    torch.cuda.synchronize()
+    ref_o, ref_l = o_g.clone(), l_g.clone()
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(s):
+        A.fwd(q, k, v, causal=True, out=o_g, lse=l_g)
+    torch.cuda.current_stream(dev).wait_stream(s)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        A.fwd(q, k, v, causal=True, out=o_g, lse=l_g)
+    torch.cuda.synchronize()
+    # wrap the eager slot ring (1024 slots) with tiny forwards
+    wt = Workload("tiny_slot", B=1, Hq=1, Hkv=1, N=128, D=64, causal=False, seed=32)
+    tq, tk, tv, _ = (x.to(dev) for x in make_inputs(wt))
+    for _ in range(1100):
+        A.fwd(tq, tk, tv)
+    torch.cuda.synchronize()
+    # replays on one stream next to eager forwards of the same shape on another
+    q2, k2, v2 = (torch.flip(x, dims=[2]).contiguous() for x in (q, k, v))
+    ref2 = A.fwd(q2, k2, v2, causal=True)
+    torch.cuda.synchronize()
+    ref2 = tuple(t.clone() for t in ref2)
+    side = torch.cuda.Stream(dev)
+    outs = []
+    for _ in range(6):
+        o_g.zero_()
+        l_g.zero_()
+        torch.cuda.synchronize()
+        g.replay()
+        with torch.cuda.stream(side):
+            for _ in range(4):
+                outs.append(A.fwd(q2, k2, v2, causal=True))
+        torch.cuda.synchronize()
+        assert A.device_status(dev) == A.FA_OK
+        assert torch.equal(o_g, ref_o) and torch.equal(l_g, ref_l)
+    for o2, l2 in outs:
+        assert torch.equal(o2, ref2[0]) and torch.equal(l2, ref2[1])

@@ -103,6 +103,21 @@ def test_backward_dq_modes(mode):
     assert r.returncode == 0, r.stdout + r.stderr
 
 
+@pytest.mark.parametrize("tile", ["m128", "m256"])
+def test_forward_tile_variants(tile):
+    """Both query-tile shapes of the bf16 forward (one CTA with 128-row MMAs;
+    a CTA pair with 256-row MMAs) match the oracle on a shape sweep, run the
+    kernel they claim to and repeat bitwise."""
+    _gpu()
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, os.path.join(here, "_fwd_tile_check.py")], env=dict(os.environ, FA_FWD_TILE=tile),
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_backward_deterministic_separate_mode():
     """The default backward has no reductions: repeated calls are bitwise equal."""
     wl = WORKLOADS["tiny"].with_(causal=True, N=700, Hq=4, Hkv=2, D=128)

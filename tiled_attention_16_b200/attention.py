@@ -121,6 +121,19 @@ def _check(t: torch.Tensor, name: str, shape, dtype=torch.bfloat16):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
+def _same_device(*tensors):
+    """The device every given tensor (None entries skipped) lives on.  The
+    library builds its tensor maps and looks up its static tables on the
+    current CUDA device, so all tensors of one call must share a device and
+    the call runs with that device made current."""
+    ts = [t for t in tensors if t is not None]
+    dev = ts[0].device
+    for t in ts[1:]:
+        if t.device != dev:
+            raise ValueError(f"all tensors must be on one device: got {dev} and {t.device}")
+    return dev
+
+
 def _dims(q, k):
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q and k must be [B, H, N, D]")
@@ -143,9 +156,11 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
         lse = torch.empty((B, Hq, N), device=q.device, dtype=torch.float32)
     _check(out, "out", (B, Hq, N, D))
     _check(lse, "lse", (B, Hq, N), torch.float32)
+    dev = _same_device(q, k, v, out, lse)
     shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
-    st = lib().fa_fwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                      lse.data_ptr(), _stream_ptr(q.device))
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_fwd")
     return out, lse
@@ -168,9 +183,11 @@ def fwd_fp8(q8: torch.Tensor, k8: torch.Tensor, v8: torch.Tensor, q_scale: float
         lse = torch.empty((B, Hq, N), device=q8.device, dtype=torch.float32)
     _check(out, "out", (B, Hq, N, D))
     _check(lse, "lse", (B, Hq, N), torch.float32)
+    dev = _same_device(q8, k8, v8, out, lse)
     shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
-    st = lib().fa_fwd_fp8(ctypes.byref(shp), q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(q_scale),
-                          float(k_scale), float(v_scale), out.data_ptr(), lse.data_ptr(), _stream_ptr(q8.device))
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd_fp8(ctypes.byref(shp), q8.data_ptr(), k8.data_ptr(), v8.data_ptr(), float(q_scale),
+                              float(k_scale), float(v_scale), out.data_ptr(), lse.data_ptr(), _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_fwd_fp8")
     return out, lse
@@ -210,8 +227,11 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tru
         workspace = torch.empty(max(nbytes, 256), device=q.device, dtype=torch.uint8)
     if workspace.device.type != "cuda" or workspace.numel() * workspace.element_size() < nbytes:
         raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
-    st = lib().fa_decode(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                         workspace.data_ptr(), workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
+    dev = _same_device(q, k, v, out, lse, workspace)
+    with torch.cuda.device(dev):
+        st = lib().fa_decode(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                             _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_decode")
     return out, lse
@@ -244,9 +264,11 @@ def bwd(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
         workspace = torch.empty(nbytes, device=q.device, dtype=torch.uint8)
     if workspace.device.type != "cuda" or workspace.numel() * workspace.element_size() < nbytes:
         raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
-    st = lib().fa_bwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
-                      workspace.numel() * workspace.element_size(), _stream_ptr(q.device))
+    dev = _same_device(q, k, v, o, do, lse, dq, dk, dv, workspace)
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), workspace.data_ptr(),
+                          workspace.numel() * workspace.element_size(), _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_bwd")
     return dq, dk, dv
@@ -269,10 +291,12 @@ def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None =
     _check(dq, "dq", (B, Hq, N, D))
     _check(dk, "dk", (B, Hkv, N, D))
     _check(dv, "dv", (B, Hkv, N, D))
+    dev = _same_device(q, k, v, o, do, lse, dq, dk, dv)
     shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
-    st = lib().fa_bwd_noalloc(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                              _stream_ptr(q.device))
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd_noalloc(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                  do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                  _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
@@ -293,9 +317,11 @@ def lse_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, 
     _check(lse_acc, "lse_acc", o_part.shape[:-1], torch.float32)
     if out is not None:
         _check(out, "out", o_part.shape)
-    st = lib().fa_lse_merge(rows, int(D), o_part.data_ptr(), lse_part.data_ptr(), o_acc.data_ptr(),
-                            lse_acc.data_ptr(), None if out is None else out.data_ptr(), 1 if first else 0,
-                            _stream_ptr(o_part.device))
+    dev = _same_device(o_part, o_acc, lse_part, lse_acc, out)
+    with torch.cuda.device(dev):
+        st = lib().fa_lse_merge(rows, int(D), o_part.data_ptr(), lse_part.data_ptr(), o_acc.data_ptr(),
+                                lse_acc.data_ptr(), None if out is None else out.data_ptr(), 1 if first else 0,
+                                _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_lse_merge")
 
@@ -309,8 +335,10 @@ def accumulate(acc: torch.Tensor, src: torch.Tensor | None, first: bool = False,
         _check(src, "src", acc.shape)
     if out is not None:
         _check(out, "out", acc.shape)
-    st = lib().fa_accumulate(acc.numel(), None if src is None else src.data_ptr(), acc.data_ptr(),
-                             None if out is None else out.data_ptr(), 1 if first else 0, _stream_ptr(acc.device))
+    dev = _same_device(acc, src, out)
+    with torch.cuda.device(dev):
+        st = lib().fa_accumulate(acc.numel(), None if src is None else src.data_ptr(), acc.data_ptr(),
+                                 None if out is None else out.data_ptr(), 1 if first else 0, _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_accumulate")
 
@@ -318,14 +346,16 @@ def accumulate(acc: torch.Tensor, src: torch.Tensor | None, first: bool = False,
 def device_status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the device status word."""
     dev = torch.device("cuda") if device is None else torch.device(device)
-    return int(lib().fa_get_device_status(_stream_ptr(dev)))
+    with torch.cuda.device(dev):   # the status word read is the current device's
+        return int(lib().fa_get_device_status(_stream_ptr(dev)))
 
 
 def selftest_wait_timeout(site: int, site2: int, device=None) -> None:
     """Launch the failure-detection self-test (fa_selftest_wait_timeout) on the
     current stream; read the outcome with device_status() and timeout_sites()."""
     dev = torch.device("cuda") if device is None else torch.device(device)
-    st = lib().fa_selftest_wait_timeout(int(site), int(site2), _stream_ptr(dev))
+    with torch.cuda.device(dev):
+        st = lib().fa_selftest_wait_timeout(int(site), int(site2), _stream_ptr(dev))
     if st != FA_OK:
         raise FAError(st, "fa_selftest_wait_timeout")
 
@@ -336,7 +366,7 @@ def timeout_sites() -> int:
 
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
                  "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode",
-                 "fa_lse_merge_kernel", "fa_accumulate_kernel")
+                 "fa_lse_merge_kernel", "fa_accumulate_kernel", "fa_fwd_pair_kernel")
 
 
 def profile_begin() -> None:

@@ -183,9 +183,7 @@ class _BwdRank:
 
     def __init__(self, ops, rank, world, q, o, do, lse, causal, scale):
         self.ops, self.q, self.o, self.do, self.scale = ops, q, o, do, scale
-        # fa_bwd wants 16-byte aligned LSE rows; the second chunk of a [2, B, H, C]
-        # shard is aligned when B*H*C is a multiple of 4, else it gets its own buffer
-        self.lse = [lse[i] if lse[i].data_ptr() % 16 == 0 else lse[i].clone() for i in (0, 1)]
+        self.lse = [lse[0], lse[1]]   # fa_bwd reads LSE one element at a time (4-byte alignment)
         self.plans = ring_plans(rank, world, causal)
         self.last = _last_use(self.plans)
         self.dq_acc = ops.empty_acc(q.shape, q)

@@ -52,6 +52,8 @@ bool make_map(CUtensorMap* map, const void* base, int BH, int N, int D, int elem
 }
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+// fp32 vectors read or written one element at a time
+bool aligned4(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 fa_status check_shape(const fa_shape* s) {
     if (!s) return FA_ERR_INVALID_ARG;
@@ -145,6 +147,27 @@ DecodePlan decode_plan(const fa_kv_shape& s) {
 
 constexpr int kNumSMs = 148;
 
+// Query tile of the bf16 forward (D = 128): "m128", 128-row MMAs on one CTA
+// (unit of 256 rows), or "m256", 256-row MMAs on a CTA pair (unit of 512
+// rows).  By default the pair is used from kPairMinN query rows on; the
+// environment variable FA_FWD_TILE=m128|m256 fixes one (read once).
+constexpr int kPairMinN = 1 << 30;
+int fwd_tile_override() {
+    static int mode = -1;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = std::getenv("FA_FWD_TILE");
+        mode = !e ? 0 : (std::strcmp(e, "m256") == 0 ? 2 : (std::strcmp(e, "m128") == 0 ? 1 : 0));
+    });
+    return mode;
+}
+bool fwd_use_pair(const fa_shape& s) {
+    if (s.D != 128) return false;
+    const int m = fwd_tile_override();
+    if (m != 0) return m == 2;
+    return s.N >= kPairMinN;
+}
+
 // dQ strategy of the backward: a separate dQ pass (default; deterministic, no
 // reductions) or the fused kernel with fp32 reductions ("atomic").  Chosen by
 // measurement; FA_DQ_MODE=atomic|separate overrides it (read once).
@@ -164,25 +187,35 @@ bool dq_separate_mode() {
 // cudaGetSymbolAddress (noalloc_scratch below).
 static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
 
-// Work-counter slots of the persistent forward.  Each launch takes the next
-// slot (round robin), so launches that may overlap on different streams use
-// different counters; the last CTA of a launch puts its slot back to zero.
-constexpr int kFwdSchedSlots = 1024;
+// Work-counter slots of the persistent forward.  A launch outside stream
+// capture takes the next slot of the first kFwdEagerSlots (round robin), so
+// launches that may overlap on different streams use different counters.  A
+// launch recorded into a CUDA graph takes a slot of its own from the rest
+// (round robin there too), so no later eager launch can share the counter a
+// graph replays with.  The last CTA of a launch puts its slot back to zero.
+constexpr int kFwdSchedSlots = 4096;
+constexpr int kFwdEagerSlots = 1024;
 static __device__ unsigned int g_fwd_sched[kFwdSchedSlots][2];
 
-fa_status fwd_sched_slot(unsigned int** out) {
+fa_status fwd_sched_slot(cudaStream_t stream, unsigned int** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return FA_ERR_CUDA;
     static std::mutex mu;
     static unsigned int* base[64] = {};
-    static unsigned int next[64] = {};
+    static unsigned int next_eager[64] = {};
+    static unsigned int next_captured[64] = {};
     std::lock_guard<std::mutex> g(mu);
     if (base[dev] == nullptr) {
         void* ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_fwd_sched) != cudaSuccess || ptr == nullptr) return FA_ERR_CUDA;
         base[dev] = static_cast<unsigned int*>(ptr);
     }
-    *out = base[dev] + 2 * (next[dev]++ % kFwdSchedSlots);
+    const unsigned int slot = (cap == cudaStreamCaptureStatusNone)
+                                  ? next_eager[dev]++ % kFwdEagerSlots
+                                  : kFwdEagerSlots + next_captured[dev]++ % (kFwdSchedSlots - kFwdEagerSlots);
+    *out = base[dev] + 2 * slot;
     return FA_OK;
 }
 
@@ -273,8 +306,9 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
     if ((st = check_device()) != FA_OK) return st;
     const fa_shape& s = *shape;
+    const bool pair = fwd_use_pair(s);
     CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
+    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D, 2, pair ? kTileN / 2 : kTileN) ||
         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D))
         return FA_ERR_CUDA;
     FwdParams p;
@@ -284,7 +318,7 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.N = s.N;
     p.causal = s.causal ? 1 : 0;
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
-    p.n_mblocks = (s.N + 2 * kTileM - 1) / (2 * kTileM);
+    p.n_mblocks = pair ? (s.N + 4 * kTileM - 1) / (4 * kTileM) : (s.N + 2 * kTileM - 1) / (2 * kTileM);
     // Query heads per scheduling group: keep the K/V streamed by the group's
     // resident CTAs within ~32 MiB of L2.
     {
@@ -296,9 +330,11 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.lse = lse;
     p.o_scale = 1.f;
     p.n_units = p.n_mblocks * s.B * s.Hq;
-    if ((st = fwd_sched_slot(&p.sched)) != FA_OK) return st;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    cudaError_t e = timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
+    p.sched = nullptr;
+    if (!pair && (st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
+    cudaError_t e = pair ? timed(10, strm, [&] { return launch_fwd_pair(tq, tk, tv, p, strm); })
+                         : timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -334,8 +370,8 @@ fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const 
     p.lse = lse;
     p.o_scale = v_scale;
     p.n_units = p.n_mblocks * s.B * s.Hq;
-    if ((st = fwd_sched_slot(&p.sched)) != FA_OK) return st;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
+    if ((st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
     cudaError_t e = timed(6, strm, [&] { return launch_fwd_fp8(tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -387,7 +423,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
                  void* stream) {
     fa_status st = check_shape(shape);
     if (st != FA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned4(lse) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
     const fa_shape& s = *shape;
@@ -463,7 +499,7 @@ fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, co
                          const void* dout, const float* lse, void* dq, void* dk, void* dv, void* stream) {
     fa_status st = check_shape(shape);
     if (st != FA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned16(lse) ||
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned4(lse) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
     if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total >

@@ -106,6 +106,11 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // ---------------------------------------------------------------------------
 // 1. preprocess
 // ---------------------------------------------------------------------------
+// Rows are handled in groups of kRowsPerIter consecutive rows per warp:
+// D/8 lanes share a row, each loading 16 bytes of O and of dO, and a warp
+// issues the loads of all its rows before reducing any of them, so every
+// warp keeps kRowsPerIter * 2 * 2D bytes in flight.  The per-row results
+// are gathered into the first lanes and written as contiguous runs.
 template <int D>
 __global__ void __launch_bounds__(256)
 fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
@@ -114,42 +119,62 @@ fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __re
                   unsigned int* __restrict__ sched) {
     // work counters of the persistent backward kernels start at zero
     if (blockIdx.x == 0 && threadIdx.x < kSchedCounters) sched[threadIdx.x] = 0u;
-    constexpr int kPer = D / 32;  // elements per lane
+    constexpr int kLanesPerRow = D / 8;                 // 16-byte loads
+    constexpr int kRowsPerLoad = 32 / kLanesPerRow;     // rows covered by one warp-wide load
+    constexpr int kUnroll = 4;
+    constexpr int kRowsPerIter = kRowsPerLoad * kUnroll; // 8 (D = 128) or 16 (D = 64); divides 128
     const int lane = threadIdx.x & 31;
+    const int sub = lane / kLanesPerRow;                // row of a load this lane serves
+    const int col = (lane % kLanesPerRow) * 8;          // first element of its 16 bytes
     const size_t warp_id = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const size_t n_warps = (static_cast<size_t>(gridDim.x) * blockDim.x) >> 5;
-    const size_t rows = static_cast<size_t>(BH) * Npad;
-    for (size_t row = warp_id; row < rows; row += n_warps) {
-        const int bh = static_cast<int>(row / Npad);
-        const int n = static_cast<int>(row - static_cast<size_t>(bh) * Npad);
-        float acc = 0.f;
-        if (n < N) {
-            const size_t base = (static_cast<size_t>(bh) * N + n) * D + lane * kPer;
-            if constexpr (kPer == 4) {
-                const uint2 a = *reinterpret_cast<const uint2*>(o + base);
-                const uint2 g = *reinterpret_cast<const uint2*>(dout + base);
-                const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-                const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+    const size_t groups = static_cast<size_t>(BH) * Npad / kRowsPerIter;
+    for (size_t grp = warp_id; grp < groups; grp += n_warps) {
+        const size_t row0 = grp * kRowsPerIter;         // never straddles a head: Npad % 128 == 0
+        const int bh = static_cast<int>(row0 / Npad);
+        const int n0 = static_cast<int>(row0 - static_cast<size_t>(bh) * Npad);
+        uint4 a[kUnroll], g[kUnroll];
 #pragma unroll
-                for (int t = 0; t < 2; ++t) {
-                    const float2 af = __bfloat1622float2(a2[t]);
-                    const float2 gf = __bfloat1622float2(g2[t]);
-                    acc = fmaf(af.x, gf.x, acc);
-                    acc = fmaf(af.y, gf.y, acc);
-                }
-            } else {
-                const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(o + base);
-                const __nv_bfloat162 g = *reinterpret_cast<const __nv_bfloat162*>(dout + base);
-                const float2 af = __bfloat1622float2(a);
-                const float2 gf = __bfloat1622float2(g);
-                acc = fmaf(af.x, gf.x, af.y * gf.y);
+        for (int u = 0; u < kUnroll; ++u) {
+            const int n = n0 + u * kRowsPerLoad + sub;
+            a[u] = make_uint4(0u, 0u, 0u, 0u);
+            g[u] = a[u];
+            if (n < N) {
+                const size_t off = (static_cast<size_t>(bh) * N + n) * D + col;
+                a[u] = *reinterpret_cast<const uint4*>(o + off);
+                g[u] = *reinterpret_cast<const uint4*>(dout + off);
             }
         }
+        float acc[kUnroll];
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) {
-            dvec[row] = acc * scale;  // the backward kernels use scale * D
-            lse2[row] = (n < N) ? lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f : INFINITY;
+        for (int u = 0; u < kUnroll; ++u) {
+            const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a[u]);
+            const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g[u]);
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 af = __bfloat1622float2(a2[t]);
+                const float2 gf = __bfloat1622float2(g2[t]);
+                s0 = fmaf(af.x, gf.x, s0);
+                s1 = fmaf(af.y, gf.y, s1);
+            }
+            acc[u] = s0 + s1;
+#pragma unroll
+            for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc[u] += __shfl_xor_sync(0xffffffffu, acc[u], off);
+        }
+        // lane j < kRowsPerIter takes row n0 + j: load u = j / kRowsPerLoad, served by lanes of sub j % kRowsPerLoad
+        const int j = lane % kRowsPerIter;
+        const int src = (j % kRowsPerLoad) * kLanesPerRow;
+        float mine = 0.f;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            const float v = __shfl_sync(0xffffffffu, acc[u], src);
+            if (j / kRowsPerLoad == u) mine = v;
+        }
+        if (lane < kRowsPerIter) {
+            const int n = n0 + lane;
+            dvec[row0 + lane] = mine * scale;   // the backward kernels use scale * D (0 on padding rows)
+            lse2[row0 + lane] = (n < N) ? lse[static_cast<size_t>(bh) * N + n] * 1.4426950408889634f : INFINITY;
         }
     }
     const size_t tid = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -588,7 +613,9 @@ cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const 
                                   cudaStream_t stream) {
     const size_t rows = static_cast<size_t>(BH) * Npad;
     const size_t dq_vec4 = dq_acc ? static_cast<size_t>(BH) * N * D / 4 : 0;
-    const int grid = grid_for(rows * 32 > dq_vec4 ? rows * 32 : dq_vec4, 256);
+    // one warp per group of 8 (D = 128) or 16 (D = 64) rows, at most 16 blocks per SM
+    const size_t warps = rows / (D == 128 ? 8 : 16);
+    const int grid = grid_for(warps * 32 > dq_vec4 ? warps * 32 : dq_vec4, 256);
     if (D == 128)
         fa_bwd_preprocess<128><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                          static_cast<const __nv_bfloat16*>(dout), lse, lse2, dvec,

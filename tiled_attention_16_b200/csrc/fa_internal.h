@@ -77,6 +77,15 @@ BwdWorkspace bwd_workspace_layout(int B, int Hq, int N, int D, bool with_dq_acc)
 cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        const FwdParams& p, cudaStream_t stream);
 
+// Forward on CTA pairs (D = 128; fa_fwd_pair.cu): work unit = 512 query rows
+// (p.n_mblocks = ceil(N / 512)), every MMA M = 256 across the pair.  tk_half
+// maps K with 64-row boxes (each CTA loads half of a key tile).  Units are
+// assigned statically; p.sched is not used.
+cudaError_t launch_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk_half, const CUtensorMap& tv,
+                            const FwdParams& p, cudaStream_t stream);
+// Pairs that can be resident at once (cached per device; -1 on error).
+int fwd_pair_max_pairs();
+
 // FP8 forward (D = 128): q/k/v maps over e4m3 bytes; p.scale_log2 already
 // includes the Q and K descales, p.o_scale is V's descale.
 cudaError_t launch_fwd_fp8(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
