@@ -116,6 +116,7 @@ KERNEL_FILES = {
     "fa_fwd_pair_kernel": ("fa_fwd_pair.cu",),
     "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu",),
     "fa_bwd_dkdv_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
+    "fa_bwd_dkdv_pair_kernel": ("fa_bwd_pair.cu", "fa_bwd.cu"),
     "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_kernel": ("fa_bwd.cu",),
     "fa_decode_split_kernel": ("fa_decode.cu",),
@@ -323,7 +324,7 @@ def run_gpu(args, wl):
     # dQ kernel 3 (S and dP recomputed, dQ).
     gemm = wl.flops_fwd() / 2
     kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_fwd_pair_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
-                    "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm}
+                    "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dkdv_pair_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm}
     tensor_k = {k: v for k, v in kms.items() if v and k in kernel_flops}
     dominant = max(tensor_k, key=lambda k: tensor_k[k])
     achieved = kernel_flops[dominant] / (tensor_k[dominant] * 1e-3) / 1e12

@@ -118,6 +118,21 @@ def test_forward_tile_variants(tile):
     assert r.returncode == 0, r.stdout + r.stderr
 
 
+@pytest.mark.parametrize("tile", ["m128", "m256"])
+def test_backward_dkdv_tile_variants(tile):
+    """Both key-block shapes of the dK/dV pass (one CTA per 128 keys; a CTA
+    pair per 256 keys with 256-row MMAs) give gradients that match the oracle
+    on a shape sweep, run the kernel they claim to and repeat bitwise."""
+    _gpu()
+    import os
+    import subprocess
+    import sys
+    here = os.path.dirname(os.path.abspath(__file__))
+    r = subprocess.run([sys.executable, os.path.join(here, "_bwd_tile_check.py")], env=dict(os.environ, FA_BWD_TILE=tile),
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
 def test_backward_deterministic_separate_mode():
     """The default backward has no reductions: repeated calls are bitwise equal."""
     wl = WORKLOADS["tiny"].with_(causal=True, N=700, Hq=4, Hkv=2, D=128)

@@ -161,6 +161,26 @@ int fwd_tile_override() {
     });
     return mode;
 }
+// Key block of the default backward's dK/dV pass (D = 128): "m128", 128-key
+// units on one CTA, or "m256", 256-key units on a CTA pair.
+// FA_BWD_TILE=m128|m256 fixes one (read once).
+constexpr int kBwdPairMinN = 1 << 30;
+int bwd_tile_override() {
+    static int mode = -1;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const char* e = std::getenv("FA_BWD_TILE");
+        mode = !e ? 0 : (std::strcmp(e, "m256") == 0 ? 2 : (std::strcmp(e, "m128") == 0 ? 1 : 0));
+    });
+    return mode;
+}
+bool bwd_use_pair(const fa_shape& s) {
+    if (s.D != 128) return false;
+    const int m = bwd_tile_override();
+    if (m != 0) return m == 2;
+    return s.N >= kBwdPairMinN;
+}
+
 bool fwd_use_pair(const fa_shape& s) {
     if (s.D != 128) return false;
     const int m = fwd_tile_override();
@@ -436,6 +456,11 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D))
         return FA_ERR_CUDA;
+    const bool pair = separate && bwd_use_pair(s);
+    CUtensorMap tq_half, tdo_half;
+    if (pair && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
+                 !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2)))
+        return FA_ERR_CUDA;
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     const int Npad = (s.N + kTileM - 1) / kTileM * kTileM;
     BwdParams p;
@@ -471,7 +496,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.dk = dk;
     p.dv = dv;
     p.sched = reinterpret_cast<unsigned int*>(wsb + ws.sched_off);
-    p.n_units_dkdv = T * s.B * s.Hkv;
+    p.n_units_dkdv = (pair ? (s.N + 2 * kTileN - 1) / (2 * kTileN) : T) * s.B * s.Hkv;
     p.n_units_dq = T * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(1, strm, [&] {
@@ -481,7 +506,9 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
                                      reinterpret_cast<unsigned int*>(wsb + ws.sched_off), strm);
     });
     if (separate) {
-        if (e == cudaSuccess) e = timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });
+        if (e == cudaSuccess)
+            e = pair ? timed(11, strm, [&] { return launch_bwd_dkdv_pair(tq, tq_half, tk, tv, tdo, tdo_half, p, strm); })
+                     : timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });
         if (e == cudaSuccess) e = timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
     } else {
         if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });

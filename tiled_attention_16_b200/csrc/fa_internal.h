@@ -107,6 +107,14 @@ cudaError_t launch_bwd_dkdv(int D, const CUtensorMap& tq, const CUtensorMap& tk,
 cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
 
+// dK/dV pass on CTA pairs (D = 128; fa_bwd_pair.cu): work unit = 256 keys
+// (p.n_units_dkdv = B * Hkv * ceil(N / 256)), every MMA M = 256 across the
+// pair.  tq_half / tdo_half map Q / dO with 64-row boxes.  Static unit
+// assignment; p.sched[0] is not used.
+cudaError_t launch_bwd_dkdv_pair(const CUtensorMap& tq, const CUtensorMap& tq_half, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdo_half,
+                                 const BwdParams& p, cudaStream_t stream);
+
 cudaError_t launch_bwd_dq_convert(const float* dq_acc, void* dq, size_t n_elems, cudaStream_t stream);
 
 // Sequence-sharded attention: log-sum-exp merge of a partial result into a
