@@ -117,6 +117,7 @@ KERNEL_FILES = {
     "fa_fwd_fp8_kernel": ("fa_fwd_fp8.cu",),
     "fa_bwd_dkdv_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_dkdv_pair_kernel": ("fa_bwd_pair.cu", "fa_bwd.cu"),
+    "fa_bwd_dq_pair_kernel": ("fa_bwd_pair.cu", "fa_bwd.cu"),
     "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_kernel": ("fa_bwd.cu",),
     "fa_decode_split_kernel": ("fa_decode.cu",),
@@ -324,7 +325,8 @@ def run_gpu(args, wl):
     # dQ kernel 3 (S and dP recomputed, dQ).
     gemm = wl.flops_fwd() / 2
     kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_fwd_pair_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
-                    "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dkdv_pair_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm}
+                    "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dkdv_pair_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm,
+                    "fa_bwd_dq_pair_kernel": 3 * gemm}
     tensor_k = {k: v for k, v in kms.items() if v and k in kernel_flops}
     dominant = max(tensor_k, key=lambda k: tensor_k[k])
     achieved = kernel_flops[dominant] / (tensor_k[dominant] * 1e-3) / 1e12
@@ -342,7 +344,8 @@ def run_gpu(args, wl):
     breakdown = {
         "fwd_ms": fwd_ms, "fwd_tflops": fwd_tf, "fwd_frac_of_peak": fwd_tf / peak_tf,
         "bwd_ms": bwd_ms, "bwd_tflops": bwd_tf, "bwd_frac_of_peak": bwd_tf / peak_tf,
-        "bwd_mode": "separate dQ pass" if kms.get("fa_bwd_dq_kernel") else "fused (fp32 dQ reductions)",
+        "bwd_mode": ("separate dQ pass" if (kms.get("fa_bwd_dq_kernel") or kms.get("fa_bwd_dq_pair_kernel"))
+                     else "fused (fp32 dQ reductions)"),
         "fwd_kernel": fwd_kernel,
         "bwd_kernels_ms": {k: v for k, v in kms.items() if v and k not in fwd_kinds},
         "bwd_preprocess_gbs": pre_bytes / (kms["fa_bwd_preprocess"] * 1e-3) / 1e9 if kms["fa_bwd_preprocess"] else None,

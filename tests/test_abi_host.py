@@ -141,7 +141,7 @@ def test_profile_hooks_without_launches():
     A.profile_begin()
     res = A.profile_end()
     assert set(res) == set(A.PROFILE_KINDS)
-    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 12
+    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 13
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
 
 

@@ -120,9 +120,10 @@ def test_forward_tile_variants(tile):
 
 @pytest.mark.parametrize("tile", ["m128", "m256"])
 def test_backward_dkdv_tile_variants(tile):
-    """Both key-block shapes of the dK/dV pass (one CTA per 128 keys; a CTA
-    pair per 256 keys with 256-row MMAs) give gradients that match the oracle
-    on a shape sweep, run the kernel they claim to and repeat bitwise."""
+    """Both block shapes of the two backward passes (one CTA per 128 keys or
+    query rows; a CTA pair per 256 with 256-row MMAs) give gradients that
+    match the oracle on a shape sweep, run the kernels they claim to and
+    repeat bitwise."""
     _gpu()
     import os
     import subprocess

@@ -367,7 +367,7 @@ def timeout_sites() -> int:
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
                  "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode",
                  "fa_lse_merge_kernel", "fa_accumulate_kernel", "fa_fwd_pair_kernel",
-                 "fa_bwd_dkdv_pair_kernel")
+                 "fa_bwd_dkdv_pair_kernel", "fa_bwd_dq_pair_kernel")
 
 
 def profile_begin() -> None:

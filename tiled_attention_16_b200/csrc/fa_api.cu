@@ -457,9 +457,11 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D))
         return FA_ERR_CUDA;
     const bool pair = separate && bwd_use_pair(s);
-    CUtensorMap tq_half, tdo_half;
+    CUtensorMap tq_half, tdo_half, tk_half, tv_half;
     if (pair && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
-                 !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2)))
+                 !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
+                 !make_map(&tk_half, k, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2) ||
+                 !make_map(&tv_half, v, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2)))
         return FA_ERR_CUDA;
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     const int Npad = (s.N + kTileM - 1) / kTileM * kTileM;
@@ -497,7 +499,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.dv = dv;
     p.sched = reinterpret_cast<unsigned int*>(wsb + ws.sched_off);
     p.n_units_dkdv = (pair ? (s.N + 2 * kTileN - 1) / (2 * kTileN) : T) * s.B * s.Hkv;
-    p.n_units_dq = T * s.B * s.Hq;
+    p.n_units_dq = (pair ? (s.N + 2 * kTileM - 1) / (2 * kTileM) : T) * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(1, strm, [&] {
         return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
@@ -509,7 +511,9 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
         if (e == cudaSuccess)
             e = pair ? timed(11, strm, [&] { return launch_bwd_dkdv_pair(tq, tq_half, tk, tv, tdo, tdo_half, p, strm); })
                      : timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });
-        if (e == cudaSuccess) e = timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
+        if (e == cudaSuccess)
+            e = pair ? timed(12, strm, [&] { return launch_bwd_dq_pair(tq, tk, tk_half, tv_half, tdo, p, strm); })
+                     : timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
     } else {
         if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
         if (e == cudaSuccess)

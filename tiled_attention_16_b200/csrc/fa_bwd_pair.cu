@@ -1,5 +1,5 @@
-// fa_bwd_pair.cu — the dK/dV pass of the tiled attention backward on CTA
-// pairs (tcgen05 cta_group::2).
+// fa_bwd_pair.cu — the dK/dV and dQ passes of the tiled attention backward
+// on CTA pairs (tcgen05 cta_group::2).
 //
 // Same mathematics as the one-CTA dK/dV pass in fa_bwd_split.cu (recompute P
 // from the saved LSE, closed-form softmax gradient dS = P o (dP - D);
@@ -485,6 +485,365 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     }
 }
 
+// ===========================================================================
+// dQ pass on CTA pairs
+// ===========================================================================
+// Unit: (batch x query head bh, 256-query block I); CTA r owns query tile
+// 2 I + r and keeps its Q and dO resident while the key tiles j stream past
+// (j <= 2 I + 1 when causal: CTA 0's rows see the last tile fully masked):
+//   S  = Q K_j^T    B = K_j split by key rows:  CTA r supplies keys [64 r, +64)
+//   dP = dO V_j^T   B = V_j split by key rows
+//   dQ += dS K_j    B = K_j split by head dim:  CTA r supplies columns [64 r, +64)
+// dS is packed bf16 over the dP block and read from tensor memory; dQ
+// accumulates in tensor memory and is written once as bf16.
+struct DqPairLayout {
+    static constexpr int kStages = 3;
+    static constexpr int kTile = kTileM * kD * 2;
+    static constexpr int kAtom = kTileM * 128;
+    static constexpr int kRowHalf = 64 * kD * 2;          // 64 key rows x 128 bf16: two 8 KB atoms
+    static constexpr int kRowAtom = 64 * 128;
+    static constexpr int kColHalf = kTileN * 64 * 2;      // 128 key rows x 64 bf16: one 16 KB atom
+    static constexpr int kQ = 0;
+    static constexpr int kDO = kQ + kTile;
+    static constexpr int kK = kDO + kTile;                // kStages x (row half, column half)
+    static constexpr int kKStage = kRowHalf + kColHalf;
+    static constexpr int kV = kK + kStages * kKStage;     // kStages x row half
+    static constexpr int kBar = kV + kStages * kRowHalf;
+    static constexpr int kNumBars = 2 + 3 * kStages + 7;
+    static constexpr int kMisc = kBar + kNumBars * 8;
+    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
+    static_assert(kBytes <= kMaxDynSmem, "pair dQ shared memory layout too large");
+};
+
+struct PairDqUnit {
+    int I, bh, kvh, n_j;
+};
+
+__device__ __forceinline__ PairDqUnit pair_dq_unit(const BwdParams& p, int T, int TI, int u) {
+    PairDqUnit w;
+    const int BH = p.B * p.Hq;
+    const int grp = u / (p.dq_heads_per_group * TI);
+    const int h0 = grp * p.dq_heads_per_group;
+    const int nh = min(p.dq_heads_per_group, BH - h0);
+    const int rr = u - grp * p.dq_heads_per_group * TI;
+    w.I = TI - 1 - rr / nh;
+    w.bh = h0 + (rr % nh);
+    const int b = w.bh / p.Hq;
+    const int h = w.bh - b * p.Hq;
+    w.kvh = b * p.Hkv + h / (p.Hq / p.Hkv);
+    w.n_j = p.causal ? min(T, 2 * w.I + 2) : T;
+    return w;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmVh,
+                      const __grid_constant__ CUtensorMap tmDO, const BwdParams p) {
+    using L = DqPairLayout;
+    constexpr int S = L::kStages;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+    if (pad + L::kBytes > static_cast<uint32_t>(L::kAlloc)) {   // same in both CTAs of the pair
+        if (threadIdx.x == 0) atomicOr(&g_status, 1u << kBPSmem);
+        return;
+    }
+    uint8_t* smem = smem_raw + pad;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+    uint64_t* q_full = bars + 0;           // leader: Q and dO of both CTAs
+    uint64_t* q_empty = bars + 1;          // both
+    uint64_t* k_full = bars + 2;           // [S] leader
+    uint64_t* v_full = k_full + S;         // [S] leader
+    uint64_t* kv_empty = v_full + S;       // [S] both
+    uint64_t* s_full = kv_empty + S;       // both
+    uint64_t* s_free = s_full + 1;         // leader: one arrival per compute warp of either CTA
+    uint64_t* dp_full = s_full + 2;        // both
+    uint64_t* ds_full = s_full + 3;        // leader
+    uint64_t* dq_done = s_full + 4;        // both
+    uint64_t* drain = s_full + 5;          // leader
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = static_cast<int>(blockIdx.x >> 1);
+    const int npairs = static_cast<int>(gridDim.x >> 1);
+    const int T = (p.N + kTileM - 1) / kTileM;
+    const int TI = (p.N + 2 * kTileM - 1) / (2 * kTileM);
+    const int n_units = p.n_units_dq;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int st = 0; st < S; ++st) {
+            mbar_init(&k_full[st], 1);
+            mbar_init(&v_full[st], 1);
+            mbar_init(&kv_empty[st], 1);
+        }
+        mbar_init(s_full, 1);
+        mbar_init(s_free, 2 * kComputeWarps);
+        mbar_init(dp_full, 1);
+        mbar_init(ds_full, 2 * kComputeWarps);
+        mbar_init(dq_done, 1);
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc_pair(tmem_slot, 512);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+    if (warp == kLoadWarp) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmKh);
+            tma_prefetch_desc(&tmVh);
+            tma_prefetch_desc(&tmDO);
+            const int rk = static_cast<int>(rank);
+            const uint32_t l_q = mapa_shared(smem_u32(q_full), 0);
+            int gj = 0;               // key tiles of the pair so far (all units)
+            int n_kv = 0, n_q = 0;    // loads issued
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int u = pair_unit_id(k, pair, npairs, n_units);
+                if (u < 0) break;
+                const PairDqUnit w = pair_dq_unit(p, T, TI, u);
+                if (k >= 1 && !(ok = mbar_wait(q_empty, (k - 1) & 1, abort_flag, kBPEmpty))) break;
+                if (rank == 0) mbar_arrive_expect_tx(q_full, 2 * 2 * L::kTile);
+                const int row0 = (2 * w.I + rk) * kTileM;
+                for (int a = 0; a < kD / 64; ++a) {
+                    tma_load_3d_pair(smem + L::kQ + a * L::kAtom, &tmQ, l_q, a * 64, row0, w.bh);
+                    tma_load_3d_pair(smem + L::kDO + a * L::kAtom, &tmDO, l_q, a * 64, row0, w.bh);
+                }
+                n_q = k + 1;
+                for (int jj = 0; jj < w.n_j; ++jj, ++gj) {
+                    const int st = gj % S;
+                    if (gj >= S && !(ok = mbar_wait(&kv_empty[st], ((gj / S) - 1) & 1, abort_flag, kBPEmpty))) break;
+                    const uint32_t lk = mapa_shared(smem_u32(&k_full[st]), 0);
+                    const uint32_t lv = mapa_shared(smem_u32(&v_full[st]), 0);
+                    uint8_t* ks = smem + L::kK + st * L::kKStage;
+                    if (rank == 0) mbar_arrive_expect_tx(&k_full[st], 2 * L::kKStage);
+                    for (int a = 0; a < kD / 64; ++a)   // key-row half (K-major): operand of S
+                        tma_load_3d_pair(ks + a * L::kRowAtom, &tmKh, lk, a * 64, jj * kTileN + 64 * rk, w.kvh);
+                    tma_load_3d_pair(ks + L::kRowHalf, &tmK, lk, 64 * rk, jj * kTileN, w.kvh);   // column half: dQ
+                    if (rank == 0) mbar_arrive_expect_tx(&v_full[st], 2 * L::kRowHalf);
+                    for (int a = 0; a < kD / 64; ++a)
+                        tma_load_3d_pair(smem + L::kV + st * L::kRowHalf + a * L::kRowAtom, &tmVh, lv, a * 64,
+                                         jj * kTileN + 64 * rk, w.kvh);
+                    n_kv = gj + 1;
+                }
+            }
+            if (rank == 0) {
+                if (n_q > 0) wait_drain(q_full, (n_q - 1) & 1, kBPDrain);
+                for (int g = (n_kv > S ? n_kv - S : 0); g < n_kv; ++g) {
+                    wait_drain(&k_full[g % S], (g / S) & 1, kBPDrain);
+                    wait_drain(&v_full[g % S], (g / S) & 1, kBPDrain);
+                }
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer (leader)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t kIdS = idesc_bf16_f32(2 * kTileM, kTileN, 0, 0);   // S, dP: K-major both
+            constexpr uint32_t kIdDQ = idesc_bf16_f32(2 * kTileM, kD, 0, 1);      // dQ: A (dS) TMEM, B MN-major
+            const uint32_t q_base = smem_u32(smem + L::kQ);
+            const uint32_t do_base = smem_u32(smem + L::kDO);
+            const uint32_t k_base = smem_u32(smem + L::kK);
+            const uint32_t v_base = smem_u32(smem + L::kV);
+            auto issue_s = [&](int st) {
+                const uint32_t kr = k_base + st * L::kKStage;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss_pair(tmem + kColS, sdesc_sw128(q_base + (kk >> 2) * L::kAtom + (kk & 3) * 32, 16, 1024),
+                                sdesc_sw128(kr + (kk >> 2) * L::kRowAtom + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
+                tc_commit_pair(s_full);
+            };
+            auto issue_dp = [&](int st) {
+                const uint32_t vr = v_base + st * L::kRowHalf;
+#pragma unroll
+                for (int kk = 0; kk < kD / 16; ++kk)
+                    mma_ss_pair(tmem + kColDP, sdesc_sw128(do_base + (kk >> 2) * L::kAtom + (kk & 3) * 32, 16, 1024),
+                                sdesc_sw128(vr + (kk >> 2) * L::kRowAtom + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
+                tc_commit_pair(dp_full);
+            };
+            bool ok = true;
+            int gj = 0;
+            for (int k = 0; ok; ++k) {
+                const int u = pair_unit_id(k, pair, npairs, n_units);
+                if (u < 0) break;
+                const int n_j = pair_dq_unit(p, T, TI, u).n_j;
+                if (!(ok = mbar_wait(q_full, k & 1, abort_flag, kBPLoad))) break;
+                if (gj > 0 && !(ok = mbar_wait_cluster(s_free, (gj - 1) & 1, abort_flag, kBPMma))) break;
+                if (!(ok = mbar_wait(&k_full[gj % S], (gj / S) & 1, abort_flag, kBPLoad))) break;
+                tc_fence_after();
+                issue_s(gj % S);
+                if (!(ok = mbar_wait(&v_full[gj % S], (gj / S) & 1, abort_flag, kBPLoad))) break;
+                tc_fence_after();
+                issue_dp(gj % S);
+                if (n_j == 1) tc_commit_pair(q_empty);
+                for (int jj = 0; jj < n_j; ++jj) {
+                    const int G = gj + jj;
+                    const int st = G % S;
+                    const int st1 = (G + 1) % S;
+                    const uint32_t ph = G & 1;
+                    if (jj + 1 < n_j) {
+                        if (!(ok = mbar_wait_cluster(s_free, ph, abort_flag, kBPMma))) break;
+                        if (!(ok = mbar_wait(&k_full[st1], ((G + 1) / S) & 1, abort_flag, kBPLoad))) break;
+                        tc_fence_after();
+                        issue_s(st1);
+                    }
+                    if (!(ok = mbar_wait_cluster(ds_full, ph, abort_flag, kBPMma))) break;
+                    tc_fence_after();
+                    const uint32_t kc = k_base + st * L::kKStage + L::kRowHalf;
+#pragma unroll
+                    for (int kk = 0; kk < kTileN / 16; ++kk)
+                        mma_ts_pair(tmem + kColDQ, tmem + kColDP + packed_col(kk),
+                                    sdesc_sw128(kc + kk * 2048, L::kColHalf, 1024), kIdDQ, (jj > 0 || kk > 0));
+                    tc_commit_pair(&kv_empty[st]);
+                    if (jj + 1 < n_j) {
+                        if (!(ok = mbar_wait(&v_full[st1], ((G + 1) / S) & 1, abort_flag, kBPLoad))) break;
+                        tc_fence_after();
+                        issue_dp(st1);
+                        if (jj + 2 == n_j) tc_commit_pair(q_empty);
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair(dq_done);
+                gj += n_j;
+            }
+            tc_commit_pair_self(drain);
+            wait_drain(drain, 0, kBPDrain);
+        }
+    } else {
+        // ------------------------------------------------------------ compute (both CTAs: P, dS)
+        const int wg = warp >> 2;
+        const int wq = warp & 3;
+        const int r = (wq << 5) + lane;  // query row of this CTA's tile = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
+        const int c0 = wg * kCols;       // this group's key columns
+        const float c = p.scale_log2;
+        const float sc = p.scale;
+        const uint32_t l_sfree = mapa_shared(smem_u32(s_free), 0);
+        const uint32_t l_ds = mapa_shared(smem_u32(ds_full), 0);
+        float pv[kCols];
+        bool ok = true;
+        int gj = 0;
+        for (int k = 0; ok; ++k) {
+            const int u = pair_unit_id(k, pair, npairs, n_units);
+            if (u < 0) break;
+            const PairDqUnit w = pair_dq_unit(p, T, TI, u);
+            const int ir = 2 * w.I + static_cast<int>(rank);   // this CTA's query tile
+            const int qrow = ir * kTileM + r;
+            const bool row_ok = qrow < p.N;                    // CTA 1's tile may lie past N (and past Npad)
+            const size_t srow = static_cast<size_t>(w.bh) * p.Npad + static_cast<size_t>(row_ok ? qrow : 0);
+            const float lse2 = row_ok ? p.lse2[srow] : INFINITY;   // +inf: P = 0
+            const float dval = row_ok ? p.dvec[srow] : 0.f;       // scale * D
+            for (int jj = 0; jj < w.n_j; ++jj) {
+                const uint32_t ph = (gj + jj) & 1;
+                ok = mbar_wait(s_full, ph, abort_flag, kBPCompute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+                {
+                    uint32_t sr[kCols / 32][32];
+#pragma unroll
+                    for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
+                    tmem_ld_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_remote(l_sfree);
+                    const float* sv = reinterpret_cast<const float*>(&sr[0][0]);
+                    const int kv0 = jj * kTileN + c0;
+                    // Masked on and after the causal diagonal tile (CTA 0 sees
+                    // the pair's last key tile entirely above its rows) and on
+                    // a partial last key tile: key columns t >= hi are zero.
+                    const float2 c2 = make_float2(c, c);
+                    const float2 nl2 = make_float2(-lse2, -lse2);
+                    static_for<0, kCols / 2>([&](auto tc) {
+                        constexpr int t = 2 * decltype(tc)::value;
+                        const float2 x = __ffma2_rn(make_float2(sv[t], sv[t + 1]), c2, nl2);
+                        pv[t] = exp2_mixed<t>(x.x);
+                        pv[t + 1] = exp2_mixed<t + 1>(x.y);
+                    });
+                    if ((p.causal && jj >= ir) || kv0 + kCols > p.N) {
+                        const int hi = min(p.N, p.causal ? qrow + 1 : p.N) - kv0;
+#pragma unroll
+                        for (int t = 0; t < kCols; ++t) pv[t] = (t < hi) ? pv[t] : 0.f;
+                    }
+                }
+                ok = mbar_wait(dp_full, ph, abort_flag, kBPCompute);
+                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int hh = 0; hh < kCols / 32; ++hh) {
+                    uint32_t dpr[32];
+                    tmem_ld32(tmem + lane_off + kColDP + c0 + hh * 32, dpr);
+                    tmem_ld_wait();
+                    uint32_t wv[16];
+                    const float2 sc2 = make_float2(sc, sc);
+                    const float2 nd2 = make_float2(-dval, -dval);
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dval = scale*D
+                        const int q0 = hh * 32 + 2 * t;
+                        const float2 gd = __ffma2_rn(
+                            make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2, nd2);
+                        const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
+                        wv[t] = pack_bf16x2(d.x, d.y);
+                    }
+                    tmem_st16(tmem + lane_off + kColDP + c0 + hh * 16, wv);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(l_ds);
+            }
+            if (!ok) break;
+            // ---- epilogue: this CTA's dQ rows (already scaled) -> bf16; the next
+            // unit's first dQ MMA overwrites them only after every compute warp's
+            // next dS arrival, which follows these loads
+            ok = mbar_wait(dq_done, k & 1, abort_flag, kBPCompute);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            tc_fence_after();
+            constexpr int kPer = kD / kGroups;
+            __nv_bfloat16* dst_row = reinterpret_cast<__nv_bfloat16*>(p.dq) +
+                                     (static_cast<size_t>(w.bh) * p.N + qrow) * kD + wg * kPer;
+#pragma unroll 1
+            for (int q = 0; q < kPer / 16; ++q) {
+                uint32_t v16[16];
+                tmem_ld16(tmem + lane_off + kColDQ + wg * kPer + q * 16, v16);
+                tmem_ld_wait();
+                uint32_t pk[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
+                if (row_ok) {
+                    uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                    dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                }
+            }
+            tc_fence_before();
+            gj += w.n_j;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, 512);
+    }
+}
+
 int dkdv_pair_max_pairs() {
     static int cache[64] = {};
     int dev = 0;
@@ -511,7 +870,47 @@ int dkdv_pair_max_pairs() {
     return cache[dev];
 }
 
+int dq_pair_max_pairs() {
+    static int cache[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+    if (cache[dev] == 0) {
+        if (cudaFuncSetAttribute(fa_bwd_dq_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 DqPairLayout::kAlloc) != cudaSuccess)
+            return -1;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * 148, 1, 1);
+        cfg.blockDim = dim3(kThreads, 1, 1);
+        cfg.dynamicSmemBytes = DqPairLayout::kAlloc;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, fa_bwd_dq_pair_kernel, &cfg) != cudaSuccess || n <= 0) return -1;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 }  // namespace
+
+cudaError_t launch_bwd_dq_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tk_half,
+                               const CUtensorMap& tv_half, const CUtensorMap& tdo, const BwdParams& p,
+                               cudaStream_t stream) {
+    if (p.n_units_dq == 0) return cudaSuccess;
+    const int max_pairs = dq_pair_max_pairs();
+    if (max_pairs <= 0) return cudaErrorInvalidConfiguration;
+    const int pairs = p.n_units_dq < max_pairs ? p.n_units_dq : max_pairs;
+    cudaError_t e = cudaFuncSetAttribute(fa_bwd_dq_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DqPairLayout::kAlloc);
+    if (e != cudaSuccess) return e;
+    fa_bwd_dq_pair_kernel<<<2 * pairs, kThreads, DqPairLayout::kAlloc, stream>>>(tq, tk, tk_half, tv_half, tdo, p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_bwd_dkdv_pair(const CUtensorMap& tq, const CUtensorMap& tq_half, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdo_half,

@@ -115,6 +115,13 @@ cudaError_t launch_bwd_dkdv_pair(const CUtensorMap& tq, const CUtensorMap& tq_ha
                                  const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdo_half,
                                  const BwdParams& p, cudaStream_t stream);
 
+// dQ pass on CTA pairs (D = 128): work unit = 256 query rows
+// (p.n_units_dq = B * Hq * ceil(N / 256)).  tk_half / tv_half map K / V with
+// 64-row boxes.  Static unit assignment; p.sched[1] is not used.
+cudaError_t launch_bwd_dq_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tk_half,
+                               const CUtensorMap& tv_half, const CUtensorMap& tdo, const BwdParams& p,
+                               cudaStream_t stream);
+
 cudaError_t launch_bwd_dq_convert(const float* dq_acc, void* dq, size_t n_elems, cudaStream_t stream);
 
 // Sequence-sharded attention: log-sum-exp merge of a partial result into a
