@@ -112,7 +112,7 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
 // warp keeps kRowsPerIter * 2 * 2D bytes in flight.  The per-row results
 // are gathered into the first lanes and written as contiguous runs.
 template <int D>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, 4)   // <= 64 registers: 32 warps per SM keep the loads in flight
 fa_bwd_preprocess(const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
                   const float* __restrict__ lse, float* __restrict__ lse2, float* __restrict__ dvec,
                   float4* __restrict__ dq_acc, size_t dq_vec4, int BH, int N, int Npad, float scale,
