@@ -240,36 +240,19 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // Arrive on a barrier of any CTA of the cluster (shared::cluster address).
+// Default (CTA-scope release) semantics: what the arrival hands over lives in
+// tensor memory and is ordered by tcgen05.wait::st + tcgen05.fence before the
+// arrival and tcgen05.fence after the wait, so no cluster-scope memory fence
+// is needed (a .release.cluster arrive costs one per compute warp and tile).
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
-    return ok != 0;
-}
-
-// mbar_wait for a barrier that threads of the other CTA arrive on (acquire at
-// cluster scope); bounded like mbar_wait.
+// mbar_wait for a barrier that threads of the other CTA arrive on; the
+// handover is tensor-memory data (see mbar_arrive_remote), so the default
+// wait suffices.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort, int site) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    unsigned long long t0 = globaltimer_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
-        if ((it & 63u) == 0) {
-            if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
-                atomicOr(&g_status, 1u << (site & 31));
-                *abort = 1;
-                return false;
-            }
-        }
-    }
+    return mbar_wait(bar, parity, abort, site);
 }
 
 // TMA load into this CTA's shared memory whose completed bytes are counted on
