@@ -351,8 +351,7 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.o_scale = 1.f;
     p.n_units = p.n_mblocks * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    p.sched = nullptr;
-    if (!pair && (st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
+    if ((st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
     cudaError_t e = pair ? timed(10, strm, [&] { return launch_fwd_pair(tq, tk, tv, p, strm); })
                          : timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -25,8 +25,9 @@
 // feed the dV / dK MMAs from tensor memory.  Loads of both CTAs count on the
 // leader's barriers; MMA completions arrive on both CTAs' barriers; each
 // compute warp of either CTA arrives once on the leader's P / dS barriers.
-// Units are assigned statically in snake order, heaviest causal blocks
-// first; every wait is bounded; no load uses multicast.
+// Units are served greedily from a work counter, heaviest causal blocks
+// first: the leader's producer takes each and publishes it in both CTAs'
+// shared memory.  Every wait is bounded; no load uses multicast.
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -67,7 +68,7 @@ struct DkdvPairLayout {
     static constexpr int kLse = kDO + 2 * kStage;         // 2 stages x 128 fp32
     static constexpr int kDvec = kLse + 2 * kTileM * 4;   // 2 stages x 128 fp32
     static constexpr int kBar = kDvec + 2 * kTileM * 4;
-    static constexpr int kNumBars = 20;
+    static constexpr int kNumBars = 24;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -116,10 +117,9 @@ __device__ __forceinline__ PairDkdvUnit pair_dkdv_unit(const BwdParams& p, int T
     return w;
 }
 
-__device__ __forceinline__ int pair_unit_id(int k, int pair, int npairs, int n_units) {
-    const int u = k * npairs + ((k & 1) ? (npairs - 1 - pair) : pair);
-    return u < n_units ? u : -1;
-}
+// Readers of each published unit id: the leader's MMA thread and compute
+// warps, the peer's producer and compute warps.
+constexpr int kUnitConsumers = 1 + kComputeWarps + 1 + kComputeWarps;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQh,
@@ -149,8 +149,11 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     uint64_t* ds_full = bars + 16;     // leader
     uint64_t* dkv_full = bars + 17;    // both
     uint64_t* drain = bars + 18;       // leader
+    uint64_t* unit_full = bars + 20;   // [2] both: the leader published a unit id in this CTA
+    uint64_t* unit_empty = bars + 22;  // [2] leader: every consumer of both CTAs has read the slot
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -179,6 +182,10 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         mbar_init(ds_full, 2 * kComputeWarps);
         mbar_init(dkv_full, 1);
         mbar_init(drain, 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&unit_full[s2], 1);
+            mbar_init(&unit_empty[s2], kUnitConsumers);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -191,6 +198,30 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256, kColDK = 384;
+
+    // Unit ring: the leader's producer takes units from the work counter
+    // (greedy, heaviest first) and publishes each id in both CTAs; every
+    // consumer reads it and releases the slot on the leader's barrier.
+    const uint32_t l_unit_empty0 = mapa_shared(smem_u32(&unit_empty[0]), 0);
+    auto take_unit = [&](int k, bool per_warp, bool& ok) -> int {
+        const int s = k & 1;
+        ok = rank == 0 ? mbar_wait(&unit_full[s], (k >> 1) & 1, abort_flag, kBPLoad)
+                       : mbar_wait_acq_cluster(&unit_full[s], (k >> 1) & 1, abort_flag, kBPLoad);
+        const int u = ok ? unit_id[s] : -1;
+        if (per_warp) __syncwarp();
+        if (!per_warp || lane == 0) mbar_arrive_remote(l_unit_empty0 + 8u * static_cast<uint32_t>(s));
+        return u;
+    };
+    // Leader's producer: publish unit `u` (-1: no more) in slot k & 1 of both CTAs.
+    auto publish_unit = [&](int k, int u) -> bool {
+        const int s = k & 1;
+        if (k >= 2 && !mbar_wait(&unit_empty[s], ((k >> 1) - 1) & 1, abort_flag, kBPEmpty)) return false;
+        unit_id[s] = u;
+        st_shared_cluster(mapa_shared(smem_u32(const_cast<int*>(&unit_id[s])), 1), u);
+        mbar_arrive(&unit_full[s]);
+        mbar_arrive_remote_release(mapa_shared(smem_u32(&unit_full[s]), 1));
+        return true;
+    };
 
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -211,9 +242,18 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             int g = 0;                         // query-tile iterations of the pair so far (all units)
             int n_q = 0, n_do = 0, n_kv = 0;   // loads issued
             bool ok = true;
+            int next = pair;   // the leader's next unit: first its pair index, then from the counter
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, n_units);
+                int u;
+                if (rank == 0) {
+                    u = next < n_units ? next : -1;
+                    if (!(ok = publish_unit(k, u))) break;
+                } else {
+                    u = take_unit(k, false, ok);
+                    if (!ok) break;
+                }
                 if (u < 0) break;
+                if (rank == 0) next = npairs + static_cast<int>(atomicAdd(p.sched + 0, 1u));
                 const PairDkdvUnit w = pair_dkdv_unit(p, T, TJ, u);
                 if (k >= 1 && !(ok = mbar_wait(kv_empty, (k - 1) & 1, abort_flag, kBPEmpty))) break;
                 if (rank == 0) mbar_arrive_expect_tx(kv_full, 2 * 2 * L::kTile);
@@ -278,8 +318,8 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
             bool ok = true;
             int g = 0;
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, n_units);
-                if (u < 0) break;
+                const int u = take_unit(k, false, ok);
+                if (!ok || u < 0) break;
                 const int n_it = pair_dkdv_unit(p, T, TJ, u).n_it;
                 if (!(ok = mbar_wait(kv_full, k & 1, abort_flag, kBPLoad))) break;
                 for (int it = 0; it < n_it; ++it) {
@@ -354,8 +394,8 @@ fa_bwd_dkdv_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_co
         bool ok = true;
         int g = 0;
         for (int k = 0; ok; ++k) {
-            const int u = pair_unit_id(k, pair, npairs, n_units);
-            if (u < 0) break;
+            const int u = take_unit(k, true, ok);
+            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
             const PairDkdvUnit w = pair_dkdv_unit(p, T, TJ, u);
             const int jr = 2 * w.J + static_cast<int>(rank);   // this CTA's 128-key block
             const int kv = jr * kTileN + r;
@@ -509,7 +549,7 @@ struct DqPairLayout {
     static constexpr int kKStage = kRowHalf + kColHalf;
     static constexpr int kV = kK + kStages * kKStage;     // kStages x row half
     static constexpr int kBar = kV + kStages * kRowHalf;
-    static constexpr int kNumBars = 2 + 3 * kStages + 7;
+    static constexpr int kNumBars = 2 + 3 * kStages + 11;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -561,8 +601,11 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     uint64_t* ds_full = s_full + 3;        // leader
     uint64_t* dq_done = s_full + 4;        // both
     uint64_t* drain = s_full + 5;          // leader
+    uint64_t* unit_full = s_full + 7;      // [2] both: the leader published a unit id in this CTA
+    uint64_t* unit_empty = s_full + 9;     // [2] leader: every consumer of both CTAs has read the slot
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -587,6 +630,10 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         mbar_init(ds_full, 2 * kComputeWarps);
         mbar_init(dq_done, 1);
         mbar_init(drain, 1);
+        for (int s2 = 0; s2 < 2; ++s2) {
+            mbar_init(&unit_full[s2], 1);
+            mbar_init(&unit_empty[s2], kUnitConsumers);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -599,6 +646,30 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256;
+
+    // Unit ring: the leader's producer takes units from the work counter
+    // (greedy, heaviest first) and publishes each id in both CTAs; every
+    // consumer reads it and releases the slot on the leader's barrier.
+    const uint32_t l_unit_empty0 = mapa_shared(smem_u32(&unit_empty[0]), 0);
+    auto take_unit = [&](int k, bool per_warp, bool& ok) -> int {
+        const int s = k & 1;
+        ok = rank == 0 ? mbar_wait(&unit_full[s], (k >> 1) & 1, abort_flag, kBPLoad)
+                       : mbar_wait_acq_cluster(&unit_full[s], (k >> 1) & 1, abort_flag, kBPLoad);
+        const int u = ok ? unit_id[s] : -1;
+        if (per_warp) __syncwarp();
+        if (!per_warp || lane == 0) mbar_arrive_remote(l_unit_empty0 + 8u * static_cast<uint32_t>(s));
+        return u;
+    };
+    // Leader's producer: publish unit `u` (-1: no more) in slot k & 1 of both CTAs.
+    auto publish_unit = [&](int k, int u) -> bool {
+        const int s = k & 1;
+        if (k >= 2 && !mbar_wait(&unit_empty[s], ((k >> 1) - 1) & 1, abort_flag, kBPEmpty)) return false;
+        unit_id[s] = u;
+        st_shared_cluster(mapa_shared(smem_u32(const_cast<int*>(&unit_id[s])), 1), u);
+        mbar_arrive(&unit_full[s]);
+        mbar_arrive_remote_release(mapa_shared(smem_u32(&unit_full[s]), 1));
+        return true;
+    };
 
     if (warp == kLoadWarp) {
         // ------------------------------------------------------------ producer (both CTAs)
@@ -613,9 +684,18 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             int gj = 0;               // key tiles of the pair so far (all units)
             int n_kv = 0, n_q = 0;    // loads issued
             bool ok = true;
+            int next = pair;
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, n_units);
+                int u;
+                if (rank == 0) {
+                    u = next < n_units ? next : -1;
+                    if (!(ok = publish_unit(k, u))) break;
+                } else {
+                    u = take_unit(k, false, ok);
+                    if (!ok) break;
+                }
                 if (u < 0) break;
+                if (rank == 0) next = npairs + static_cast<int>(atomicAdd(p.sched + 1, 1u));
                 const PairDqUnit w = pair_dq_unit(p, T, TI, u);
                 if (k >= 1 && !(ok = mbar_wait(q_empty, (k - 1) & 1, abort_flag, kBPEmpty))) break;
                 if (rank == 0) mbar_arrive_expect_tx(q_full, 2 * 2 * L::kTile);
@@ -678,8 +758,8 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
             bool ok = true;
             int gj = 0;
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, n_units);
-                if (u < 0) break;
+                const int u = take_unit(k, false, ok);
+                if (!ok || u < 0) break;
                 const int n_j = pair_dq_unit(p, T, TI, u).n_j;
                 if (!(ok = mbar_wait(q_full, k & 1, abort_flag, kBPLoad))) break;
                 if (gj > 0 && !(ok = mbar_wait_cluster(s_free, (gj - 1) & 1, abort_flag, kBPMma))) break;
@@ -738,8 +818,8 @@ fa_bwd_dq_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_cons
         bool ok = true;
         int gj = 0;
         for (int k = 0; ok; ++k) {
-            const int u = pair_unit_id(k, pair, npairs, n_units);
-            if (u < 0) break;
+            const int u = take_unit(k, true, ok);
+            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
             const PairDqUnit w = pair_dq_unit(p, T, TI, u);
             const int ir = 2 * w.I + static_cast<int>(rank);   // this CTA's query tile
             const int qrow = ir * kTileM + r;

@@ -33,8 +33,9 @@
 //     (commit with a CTA mask), which release the stages for both producers
 //     and hand S and O to both CTAs' softmax warps;
 //   * each softmax warp of either CTA arrives once on the leader's P barrier.
-// Units are assigned statically (snake order over the pairs, heaviest causal
-// blocks first), so the two CTAs agree on the sequence without exchanging it.
+// Units are served greedily (heaviest causal blocks first): the leader's
+// producer takes each from the launch's counter slot and publishes it in both
+// CTAs' shared memory; the peer's producer and softmax warps read it there.
 // Every wait is bounded; no load uses multicast.
 #include "fa_internal.h"
 #include "sm100.cuh"
@@ -48,6 +49,9 @@ namespace {
 constexpr int kThreads = 320;
 constexpr int kD = 128;
 constexpr int kStages = 3;
+// Readers of each published unit id: the leader's MMA thread and 8 softmax
+// warps, the peer's producer and 8 softmax warps.
+constexpr int kUnitConsumers = 1 + 8 + 1 + 8;
 constexpr float kRescaleThreshold = 8.0f;
 
 enum PairSite { kPSiteQ = 0, kPSiteK = 1, kPSiteV = 2, kPSiteKVEmpty = 3, kPSiteS = 4, kPSiteP = 5, kPSiteO = 6,
@@ -63,7 +67,7 @@ struct PairLayout {
     static constexpr int kK = kQ + 2 * kQTile;               // kStages halves
     static constexpr int kV = kK + kStages * kKHalf;
     static constexpr int kBar = kV + kStages * kVHalf;
-    static constexpr int kNumBars = 2 + 3 * kStages + 3 * 2 + 1;   // q full/empty, k/v full + empty, s/p/o, drain
+    static constexpr int kNumBars = 2 + 3 * kStages + 3 * 2 + 1 + 4;   // q, k/v ring, s/p/o, drain, unit ring
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -129,12 +133,6 @@ __device__ __forceinline__ PairUnit pair_unit(const FwdParams& p, int u) {
     return w;
 }
 
-// k-th unit of pair `pair` in snake order over `npairs` pairs (-1: none left).
-__device__ __forceinline__ int pair_unit_id(int k, int pair, int npairs, int n_units) {
-    const int u = k * npairs + ((k & 1) ? (npairs - 1 - pair) : pair);
-    return u < n_units ? u : -1;
-}
-
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -152,8 +150,11 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     uint64_t* p_full = s_full + 2;               // [2] leader: one arrival per softmax warp of either CTA
     uint64_t* o_full = p_full + 2;               // [2] both
     uint64_t* drain = o_full + 2;                // leader
+    uint64_t* unit_full = drain + 1;             // [2] both: the leader published a unit id in this CTA
+    uint64_t* unit_empty = drain + 3;            // [2] leader: every consumer of both CTAs has read the slot
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+    volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);   // [2]
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -175,6 +176,10 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mbar_init(&o_full[s], 1);
         }
         mbar_init(drain, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&unit_full[s], 1);
+            mbar_init(&unit_empty[s], kUnitConsumers);
+        }
         *abort_flag = 0;
         fence_mbar_init();
     }
@@ -188,6 +193,21 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
+    // Unit ring: the leader's producer takes units from the launch's counter
+    // (greedy, heaviest first) and publishes each id in both CTAs; every
+    // consumer (the leader's MMA thread, both CTAs' softmax warps and the
+    // peer's producer) reads it and releases the slot on the leader's barrier.
+    const uint32_t l_unit_empty0 = mapa_shared(smem_u32(&unit_empty[0]), 0);
+    auto take_unit = [&](int k, bool per_warp, bool& ok) -> int {
+        const int s = k & 1;
+        ok = rank == 0 ? mbar_wait(&unit_full[s], (k >> 1) & 1, abort_flag, kPSiteQ)
+                       : mbar_wait_acq_cluster(&unit_full[s], (k >> 1) & 1, abort_flag, kPSiteQ);
+        const int u = ok ? unit_id[s] : -1;
+        if (per_warp) __syncwarp();
+        if (!per_warp || lane == 0) mbar_arrive_remote(l_unit_empty0 + 8u * static_cast<uint32_t>(s));
+        return u;
+    };
+
     if (warp == 9) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
@@ -198,9 +218,23 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             int gk = 0;               // K/V tiles of this pair so far (all units)
             int n_kv = 0, n_q = 0;    // loads issued by this CTA
             bool ok = true;
+            int next = pair;          // the leader's next unit: first its pair index, then from the counter
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, p.n_units);
+                int u;
+                if (rank == 0) {
+                    const int s = k & 1;
+                    if (k >= 2 && !(ok = mbar_wait(&unit_empty[s], ((k >> 1) - 1) & 1, abort_flag, kPSiteKVEmpty))) break;
+                    u = next < p.n_units ? next : -1;
+                    unit_id[s] = u;
+                    st_shared_cluster(mapa_shared(smem_u32(const_cast<int*>(&unit_id[s])), 1), u);
+                    mbar_arrive(&unit_full[s]);
+                    mbar_arrive_remote_release(mapa_shared(smem_u32(&unit_full[s]), 1));
+                } else {
+                    u = take_unit(k, false, ok);
+                    if (!ok) break;
+                }
                 if (u < 0) break;
+                if (rank == 0) next = npairs + static_cast<int>(atomicAdd(p.sched, 1u));
                 const PairUnit w = pair_unit(p, u);
                 const int nsub = w.nkv1 > 0 ? 2 : 1;
                 if (k >= 1 && !(ok = mbar_wait(q_empty, (k - 1) & 1, abort_flag, kPSiteKVEmpty))) break;
@@ -268,8 +302,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             int gk = 0;                // K/V tiles consumed (all units)
             int c0 = 0, c1 = 0;        // S tiles issued for query tile 0 / 1 (all units)
             for (int k = 0; ok; ++k) {
-                const int u = pair_unit_id(k, pair, npairs, p.n_units);
-                if (u < 0) break;
+                const int u = take_unit(k, false, ok);
+                if (!ok || u < 0) break;
                 const PairUnit w = pair_unit(p, u);
                 const int nkv[2] = {w.nkv0, w.nkv1};
                 const int n_iter = w.n_iter;
@@ -338,8 +372,8 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         int cs = 0;      // S tiles of this query tile so far (all units)
         int uo = 0;      // units in which this query tile was active
         for (int k = 0; ok; ++k) {
-            const int u = pair_unit_id(k, pair, npairs, p.n_units);
-            if (u < 0) break;
+            const int u = take_unit(k, true, ok);
+            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
             const PairUnit w = pair_unit(p, u);
             const int nkv_s = s == 0 ? w.nkv0 : w.nkv1;
             const int row0 = w.m0 + 2 * kTileM * s + kTileM * static_cast<int>(rank);   // this CTA's first row
@@ -458,6 +492,15 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc_pair(tmem, 512);
+    }
+    // the last CTA to leave returns the launch's counter slot to zero
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+            p.sched[0] = 0u;
+            p.sched[1] = 0u;
+            __threadfence();
+        }
     }
 }
 

@@ -80,7 +80,7 @@ cudaError_t launch_fwd(int D, const CUtensorMap& tq, const CUtensorMap& tk, cons
 // Forward on CTA pairs (D = 128; fa_fwd_pair.cu): work unit = 512 query rows
 // (p.n_mblocks = ceil(N / 512)), every MMA M = 256 across the pair.  tk_half
 // maps K with 64-row boxes (each CTA loads half of a key tile).  Units are
-// assigned statically; p.sched is not used.
+// served greedily from the counter slot p.sched, as in the one-CTA kernel.
 cudaError_t launch_fwd_pair(const CUtensorMap& tq, const CUtensorMap& tk_half, const CUtensorMap& tv,
                             const FwdParams& p, cudaStream_t stream);
 // Pairs that can be resident at once (cached per device; -1 on error).
@@ -109,15 +109,15 @@ cudaError_t launch_bwd_dq(int D, const CUtensorMap& tq, const CUtensorMap& tk, c
 
 // dK/dV pass on CTA pairs (D = 128; fa_bwd_pair.cu): work unit = 256 keys
 // (p.n_units_dkdv = B * Hkv * ceil(N / 256)), every MMA M = 256 across the
-// pair.  tq_half / tdo_half map Q / dO with 64-row boxes.  Static unit
-// assignment; p.sched[0] is not used.
+// pair.  tq_half / tdo_half map Q / dO with 64-row boxes.  Units are served
+// greedily from the counter p.sched[0].
 cudaError_t launch_bwd_dkdv_pair(const CUtensorMap& tq, const CUtensorMap& tq_half, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& tdo, const CUtensorMap& tdo_half,
                                  const BwdParams& p, cudaStream_t stream);
 
 // dQ pass on CTA pairs (D = 128): work unit = 256 query rows
 // (p.n_units_dq = B * Hq * ceil(N / 256)).  tk_half / tv_half map K / V with
-// 64-row boxes.  Static unit assignment; p.sched[1] is not used.
+// 64-row boxes.  Units are served greedily from the counter p.sched[1].
 cudaError_t launch_bwd_dq_pair(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tk_half,
                                const CUtensorMap& tv_half, const CUtensorMap& tdo, const BwdParams& p,
                                cudaStream_t stream);
