@@ -241,10 +241,10 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * tiles), 11 backward dK/dV kernel on CTA pairs (256-key blocks), 12
  * backward dQ kernel on CTA pairs (256-query blocks) (FA_PROFILE_KINDS;
  * fa_fwd uses 0, or 10 when the environment variable FA_FWD_TILE=m256 selects
- * the CTA-pair kernel for D = 128; fa_bwd uses 1, 4, 5 by default, 1, 11, 12
- * when FA_BWD_TILE=m256 selects the CTA-pair passes for D = 128, and 1, 2, 3
- * when FA_DQ_MODE=atomic selects the fused kernel).  Events are host-created
- * objects; no device memory is allocated. */
+ * the CTA-pair kernel for D = 128; fa_bwd uses 1, 4, 5 by default,
+ * FA_BWD_TILE=m256 selects the CTA-pair passes (1, 11, 12) for D = 128, and
+ * FA_DQ_MODE=atomic the fused kernel (1, 2, 3)).  Events are host-created objects; no device
+ * memory is allocated. */
 #define FA_PROFILE_KINDS 13
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);

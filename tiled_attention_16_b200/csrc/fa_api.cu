@@ -161,9 +161,11 @@ int fwd_tile_override() {
     });
     return mode;
 }
-// Key block of the default backward's dK/dV pass (D = 128): "m128", 128-key
-// units on one CTA, or "m256", 256-key units on a CTA pair.
-// FA_BWD_TILE=m128|m256 fixes one (read once).
+// Block of the default backward's two passes (D = 128): "m128", 128 keys
+// (dK/dV pass) or 128 query rows (dQ pass) per CTA, or "m256", 256 per CTA
+// pair.  FA_BWD_TILE=m128|m256 fixes both (read once).  By measurement both
+// passes run on one CTA by default (the pairs were equal or slower on every
+// workload measured); kBwdPairMinN is where the dQ pass would switch.
 constexpr int kBwdPairMinN = 1 << 30;
 int bwd_tile_override() {
     static int mode = -1;
@@ -174,7 +176,11 @@ int bwd_tile_override() {
     });
     return mode;
 }
-bool bwd_use_pair(const fa_shape& s) {
+bool bwd_dkdv_use_pair(const fa_shape& s) {
+    if (s.D != 128) return false;
+    return bwd_tile_override() == 2;
+}
+bool bwd_dq_use_pair(const fa_shape& s) {
     if (s.D != 128) return false;
     const int m = bwd_tile_override();
     if (m != 0) return m == 2;
@@ -455,12 +461,14 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D))
         return FA_ERR_CUDA;
-    const bool pair = separate && bwd_use_pair(s);
+    const bool pair_dkdv = separate && bwd_dkdv_use_pair(s);
+    const bool pair_dq = separate && bwd_dq_use_pair(s);
     CUtensorMap tq_half, tdo_half, tk_half, tv_half;
-    if (pair && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
-                 !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
-                 !make_map(&tk_half, k, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2) ||
-                 !make_map(&tv_half, v, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2)))
+    if (pair_dkdv && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
+                      !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2)))
+        return FA_ERR_CUDA;
+    if (pair_dq && (!make_map(&tk_half, k, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2) ||
+                    !make_map(&tv_half, v, s.B * s.Hkv, s.N, s.D, 2, kTileN / 2)))
         return FA_ERR_CUDA;
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     const int Npad = (s.N + kTileM - 1) / kTileM * kTileM;
@@ -497,8 +505,8 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.dk = dk;
     p.dv = dv;
     p.sched = reinterpret_cast<unsigned int*>(wsb + ws.sched_off);
-    p.n_units_dkdv = (pair ? (s.N + 2 * kTileN - 1) / (2 * kTileN) : T) * s.B * s.Hkv;
-    p.n_units_dq = (pair ? (s.N + 2 * kTileM - 1) / (2 * kTileM) : T) * s.B * s.Hq;
+    p.n_units_dkdv = (pair_dkdv ? (s.N + 2 * kTileN - 1) / (2 * kTileN) : T) * s.B * s.Hkv;
+    p.n_units_dq = (pair_dq ? (s.N + 2 * kTileM - 1) / (2 * kTileM) : T) * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     cudaError_t e = timed(1, strm, [&] {
         return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
@@ -508,10 +516,10 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     });
     if (separate) {
         if (e == cudaSuccess)
-            e = pair ? timed(11, strm, [&] { return launch_bwd_dkdv_pair(tq, tq_half, tk, tv, tdo, tdo_half, p, strm); })
+            e = pair_dkdv ? timed(11, strm, [&] { return launch_bwd_dkdv_pair(tq, tq_half, tk, tv, tdo, tdo_half, p, strm); })
                      : timed(4, strm, [&] { return launch_bwd_dkdv(s.D, tq, tk, tv, tdo, p, strm); });
         if (e == cudaSuccess)
-            e = pair ? timed(12, strm, [&] { return launch_bwd_dq_pair(tq, tk, tk_half, tv_half, tdo, p, strm); })
+            e = pair_dq ? timed(12, strm, [&] { return launch_bwd_dq_pair(tq, tk, tk_half, tv_half, tdo, p, strm); })
                      : timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
     } else {
         if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
