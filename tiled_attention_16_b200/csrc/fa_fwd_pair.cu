@@ -420,19 +420,21 @@ fa_fwd_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const float2 c2 = make_float2(c, c);
                 const float2 nm2 = make_float2(-msub, -msub);
                 float2 ls2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                // four quarters of 32 columns, each packed into 16 TMEM columns as
+                // soon as it is formed (few registers beyond the S row stay live)
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t pk[32];
+                for (int qtr = 0; qtr < 4; ++qtr) {
+                    uint32_t pk[16];
 #pragma unroll
-                    for (int t = 0; t < 32; ++t) {
-                        const int cix = half * 64 + 2 * t;
+                    for (int t = 0; t < 16; ++t) {
+                        const int cix = qtr * 32 + 2 * t;
                         const float2 x = __ffma2_rn(make_float2(sv[cix], sv[cix + 1]), c2, nm2);
                         const float p0 = ex2(x.x);
                         const float p1 = ex2(x.y);
                         ls2[t & 1] = __fadd2_rn(ls2[t & 1], make_float2(p0, p1));
                         pk[t] = pack_bf16x2(p0, p1);
                     }
-                    tmem_st32(tS + half * 32, pk);
+                    tmem_st16(tS + qtr * 16, pk);
                 }
                 l += (ls2[0].x + ls2[0].y) + (ls2[1].x + ls2[1].y);
                 if (rescale && j > 0) {
