@@ -197,6 +197,48 @@ FA_API fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void
 FA_API fa_status fa_lse_merge(long long rows, int D, const void* o_part, const float* lse_part, float* o_acc,
                               float* lse_acc, void* o_out, int first, void* stream);
 
+/* Fused forms of the per-pair steps above (the same results, fewer passes
+ * over memory):
+ *
+ * fa_fwd_merge computes what fa_fwd computes for q over (k, v) and folds it,
+ * inside the forward kernel's epilogue, into a running fp32 result by the
+ * log-sum-exp rule of fa_lse_merge instead of writing o and lse:
+ *   o_acc   fp32 [B,Hq,N,D]  running result, normalised (in/out)
+ *   lse_acc fp32 [B,Hq,N]    its natural-log LSE (in/out)
+ *   o_out   bf16 [B,Hq,N,D]  optional (NULL allowed): also receives the merged result
+ *   first   nonzero: o_acc / lse_acc are not read and are set from this call
+ * The one-CTA forward kernel runs it whatever FA_FWD_TILE says.  q, k, v as
+ * for fa_fwd; o_acc, o_out 16-byte aligned, lse_acc 4-byte aligned; errors
+ * and asynchrony as for fa_fwd. */
+FA_API fa_status fa_fwd_merge(const fa_shape* shape, const void* q, const void* k, const void* v, float* o_acc,
+                              float* lse_acc, void* o_out, int first, void* stream);
+
+/* fa_bwd split in two for a query block whose backward runs against several
+ * key blocks:
+ *
+ * fa_bwd_stats writes the row statistics of the backward (LSE in log2 units
+ * and scale * rowsum(dO o O), the preprocess of fa_bwd) for (o, dout, lse)
+ * into `workspace` (at least fa_bwd_workspace_bytes(shape) bytes, 256-byte
+ * aligned) and launches nothing else.
+ *
+ * fa_bwd_accumulate then runs the two gradient passes of fa_bwd on those
+ * statistics and ADDS the gradients into fp32 sums instead of writing bf16:
+ *   dq_acc fp32 [B,Hq,N,D], dk_acc and dv_acc fp32 [B,Hkv,N,D]  (in/out, 16-byte aligned)
+ *   flags  FA_ACC_DQ_FIRST: dq_acc is overwritten, not added to;
+ *          FA_ACC_DKV_FIRST: the same for dk_acc and dv_acc.
+ * The workspace must hold the statistics fa_bwd_stats wrote for the same
+ * shape and the same o, dout and lse; its work counters are reset here.  q,
+ * k, v, dout as for fa_bwd (dout is read again by the passes).  Always the
+ * one-CTA passes with the separate dQ pass (whatever FA_BWD_TILE and
+ * FA_DQ_MODE say).  Errors and asynchrony as for fa_bwd. */
+#define FA_ACC_DQ_FIRST 1
+#define FA_ACC_DKV_FIRST 2
+FA_API fa_status fa_bwd_stats(const fa_shape* shape, const void* o, const void* dout, const float* lse,
+                              void* workspace, size_t workspace_bytes, void* stream);
+FA_API fa_status fa_bwd_accumulate(const fa_shape* shape, const void* q, const void* k, const void* v,
+                                   const void* dout, float* dq_acc, float* dk_acc, float* dv_acc, int flags,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
 /* Gradient accumulation: acc = (first ? 0 : acc) + src, elementwise over n
  * elements (src bf16, acc fp32; src NULL adds nothing), and out = bf16(acc)
  * when out is not NULL.  n >= 0 and a multiple of 8; device pointers 16-byte

@@ -40,6 +40,21 @@ class OracleOps:
         if out is not None:
             out.copy_(o_acc)
 
+    def fwd_merge(self, q, k, v, causal_flag, scale, o_acc, lse_acc, first, out=None):
+        o_p, lse_p = self.fwd(q, k, v, causal_flag, scale)
+        self.merge(o_acc, lse_acc, o_p, lse_p, first, out)
+
+    def bwd_prepare(self, o, do, lse, scale):
+        # the oracle's block backward takes the full rows' output and LSE
+        return (o, lse)
+
+    def bwd_accumulate(self, q, k, v, do, prep, causal_flag, scale, dq_acc, dk_acc, dv_acc, first_dq, first_dkv):
+        o, lse = prep
+        dq, dk, dv = self.bwd(q, k, v, o, do, lse, causal_flag, scale)
+        self.accumulate(dq_acc, dq, first_dq)
+        self.accumulate(dk_acc, dk, first_dkv)
+        self.accumulate(dv_acc, dv, first_dkv)
+
     def accumulate(self, acc, src, first, out=None):
         if first:
             acc.zero_()

@@ -21,7 +21,8 @@ def test_exports_every_declared_symbol():
     assert set(names) == {"fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_get_device_status",
                           "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
                           "fa_bwd_noalloc", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes",
-                          "fa_lse_merge", "fa_accumulate", "fa_selftest_wait_timeout"}
+                          "fa_lse_merge", "fa_accumulate", "fa_selftest_wait_timeout", "fa_fwd_merge",
+                          "fa_bwd_stats", "fa_bwd_accumulate"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -269,3 +270,41 @@ def test_merge_and_accumulate_valid_calls_fail_cleanly_without_gpu():
 def test_selftest_rejects_bad_sites_before_launch():
     for a, b in ((-1, 0), (0, 32), (5, 5), (40, 1)):
         assert A.lib().fa_selftest_wait_timeout(a, b, None) == A.FA_ERR_INVALID_ARG
+
+
+# ---- fused sequence-sharding steps (fa_fwd_merge, fa_bwd_stats, fa_bwd_accumulate)
+def test_fwd_merge_host_checks():
+    f = lambda shp, **kw: A.lib().fa_fwd_merge(  # noqa: E731
+        None if shp is None else ctypes.byref(shp), kw.get("q", P), kw.get("k", P), kw.get("v", P),
+        kw.get("o_acc", P), kw.get("lse_acc", P), kw.get("o_out", None), 0, None)
+    assert f(None) == A.FA_ERR_INVALID_ARG
+    assert f(shape(N=0)) == A.FA_ERR_INVALID_ARG
+    assert f(shape(D=96)) == A.FA_ERR_UNSUPPORTED
+    for which in ("q", "k", "v", "o_acc"):
+        assert f(shape(), **{which: P + 8}) == A.FA_ERR_INVALID_ARG
+        assert f(shape(), **{which: 0}) == A.FA_ERR_INVALID_ARG
+    assert f(shape(), lse_acc=P + 2) == A.FA_ERR_INVALID_ARG    # fp32 vector: 4-byte alignment
+    assert f(shape(), o_out=P + 8) == A.FA_ERR_INVALID_ARG
+
+
+def test_bwd_stats_and_accumulate_host_checks():
+    s = shape()
+    need = A.lib().fa_bwd_workspace_bytes(ctypes.byref(s))
+    st = lambda shp, ws=P, nb=need, **kw: A.lib().fa_bwd_stats(  # noqa: E731
+        None if shp is None else ctypes.byref(shp), kw.get("o", P), kw.get("do", P), kw.get("lse", P), ws, nb, None)
+    assert st(None) == A.FA_ERR_INVALID_ARG
+    assert st(shape(D=96)) == A.FA_ERR_UNSUPPORTED
+    assert st(s, o=P + 8) == A.FA_ERR_INVALID_ARG
+    assert st(s, lse=P + 2) == A.FA_ERR_INVALID_ARG
+    assert st(s, ws=0) == A.FA_ERR_INVALID_ARG
+    assert st(s, ws=P + 16) == A.FA_ERR_INVALID_ARG          # not 256-byte aligned
+    assert st(s, nb=need - 1) == A.FA_ERR_INVALID_ARG
+    acc = lambda shp, flags=0, ws=P, nb=need, **kw: A.lib().fa_bwd_accumulate(  # noqa: E731
+        None if shp is None else ctypes.byref(shp), kw.get("q", P), kw.get("k", P), kw.get("v", P), kw.get("do", P),
+        kw.get("dq", P), kw.get("dk", P), kw.get("dv", P), flags, ws, nb, None)
+    assert acc(None) == A.FA_ERR_INVALID_ARG
+    assert acc(s, flags=4) == A.FA_ERR_INVALID_ARG           # unknown flag bit
+    for which in ("q", "k", "v", "do", "dq", "dk", "dv"):
+        assert acc(s, **{which: P + 8}) == A.FA_ERR_INVALID_ARG
+    assert acc(s, ws=0) == A.FA_ERR_INVALID_ARG
+    assert acc(s, nb=need - 1) == A.FA_ERR_INVALID_ARG

@@ -79,6 +79,12 @@ def lib() -> ctypes.CDLL:
         L.fa_lse_merge.restype = ctypes.c_int
         L.fa_accumulate.argtypes = [ll, vp, vp, vp, ctypes.c_int, vp]
         L.fa_accumulate.restype = ctypes.c_int
+        L.fa_fwd_merge.argtypes = [shp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
+        L.fa_fwd_merge.restype = ctypes.c_int
+        L.fa_bwd_stats.argtypes = [shp, vp, vp, vp, vp, sz, vp]
+        L.fa_bwd_stats.restype = ctypes.c_int
+        L.fa_bwd_accumulate.argtypes = [shp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp, sz, vp]
+        L.fa_bwd_accumulate.restype = ctypes.c_int
         L.fa_selftest_wait_timeout.argtypes = [ctypes.c_int, ctypes.c_int, vp]
         L.fa_selftest_wait_timeout.restype = ctypes.c_int
         L.fa_profile_begin.argtypes = []
@@ -300,6 +306,85 @@ def bwd_noalloc(q, k, v, o, do, lse, causal: bool = False, scale: float | None =
     if st != FA_OK:
         raise FAError(st, "fa_bwd_noalloc")
     return dq, dk, dv
+
+
+FA_ACC_DQ_FIRST, FA_ACC_DKV_FIRST = 1, 2
+
+
+def fwd_merge(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o_acc: torch.Tensor, lse_acc: torch.Tensor,
+              causal: bool = False, scale: float | None = None, first: bool = False,
+              out: torch.Tensor | None = None) -> None:
+    """Attention of q over (k, v), folded into the running fp32 result
+    (o_acc [B,Hq,N,D], lse_acc [B,Hq,N]) in place by the log-sum-exp rule
+    inside the forward kernel (fa_fwd_merge); first=True sets it from this
+    call; `out` (bf16) also receives the merged result."""
+    B, Hq, Hkv, N, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(q, "q", (B, Hq, N, D))
+    _check(k, "k", (B, Hkv, N, D))
+    _check(v, "v", (B, Hkv, N, D))
+    _check(o_acc, "o_acc", (B, Hq, N, D), torch.float32)
+    _check(lse_acc, "lse_acc", (B, Hq, N), torch.float32)
+    if out is not None:
+        _check(out, "out", (B, Hq, N, D))
+    dev = _same_device(q, k, v, o_acc, lse_acc, out)
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    with torch.cuda.device(dev):
+        st = lib().fa_fwd_merge(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), o_acc.data_ptr(),
+                                lse_acc.data_ptr(), None if out is None else out.data_ptr(), 1 if first else 0,
+                                _stream_ptr(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_fwd_merge")
+
+
+def bwd_stats(o: torch.Tensor, do: torch.Tensor, lse: torch.Tensor, causal: bool = False, scale: float | None = None,
+              workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Row statistics of the backward for (o, do, lse) written into a
+    workspace (fa_bwd_stats); returns the workspace for bwd_accumulate."""
+    B, Hq, N, D = o.shape
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    _check(o, "o", (B, Hq, N, D))
+    _check(do, "do", (B, Hq, N, D))
+    _check(lse, "lse", (B, Hq, N), torch.float32)
+    shp = make_shape(B, Hq, Hq, N, D, scale, causal)
+    nbytes = int(lib().fa_bwd_workspace_bytes(ctypes.byref(shp)))
+    if workspace is None:
+        workspace = torch.empty(nbytes, device=o.device, dtype=torch.uint8)
+    if workspace.device.type != "cuda" or workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError(f"workspace must be a CUDA buffer of at least {nbytes} bytes")
+    dev = _same_device(o, do, lse, workspace)
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd_stats(ctypes.byref(shp), o.data_ptr(), do.data_ptr(), lse.data_ptr(), workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream_ptr(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_stats")
+    return workspace
+
+
+def bwd_accumulate(q, k, v, do, workspace: torch.Tensor, dq_acc: torch.Tensor, dk_acc: torch.Tensor,
+                   dv_acc: torch.Tensor, causal: bool = False, scale: float | None = None, first_dq: bool = False,
+                   first_dkv: bool = False) -> None:
+    """Gradients of (q, k, v) on the statistics that bwd_stats left in
+    `workspace`, added into fp32 sums in place (fa_bwd_accumulate); the first
+    flags overwrite instead of adding."""
+    B, Hq, Hkv, N, D = _dims(q, k)
+    scale = 1.0 / math.sqrt(D) if scale is None else float(scale)
+    for t, name, shape in ((q, "q", (B, Hq, N, D)), (k, "k", (B, Hkv, N, D)), (v, "v", (B, Hkv, N, D)),
+                           (do, "do", (B, Hq, N, D))):
+        _check(t, name, shape)
+    _check(dq_acc, "dq_acc", (B, Hq, N, D), torch.float32)
+    _check(dk_acc, "dk_acc", (B, Hkv, N, D), torch.float32)
+    _check(dv_acc, "dv_acc", (B, Hkv, N, D), torch.float32)
+    dev = _same_device(q, k, v, do, workspace, dq_acc, dk_acc, dv_acc)
+    shp = make_shape(B, Hq, Hkv, N, D, scale, causal)
+    flags = (FA_ACC_DQ_FIRST if first_dq else 0) | (FA_ACC_DKV_FIRST if first_dkv else 0)
+    with torch.cuda.device(dev):
+        st = lib().fa_bwd_accumulate(ctypes.byref(shp), q.data_ptr(), k.data_ptr(), v.data_ptr(), do.data_ptr(),
+                                     dq_acc.data_ptr(), dk_acc.data_ptr(), dv_acc.data_ptr(), flags,
+                                     workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                                     _stream_ptr(dev))
+    if st != FA_OK:
+        raise FAError(st, "fa_bwd_accumulate")
 
 
 def lse_merge(o_acc: torch.Tensor, lse_acc: torch.Tensor, o_part: torch.Tensor, lse_part: torch.Tensor,

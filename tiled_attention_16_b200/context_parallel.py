@@ -15,18 +15,20 @@ Forward on rank r.  For s = 0 .. R-1 the rank holds the K/V shard of rank
 src = (r - s) mod R.  Each of its query chunks a meets each key chunk b of
 that shard: b < a is a full (unmasked) square attention, b == a the causal
 diagonal, b > a is skipped (non-causal attention takes every pair).  Every
-pair is one fa_fwd call on (C x C) chunks; its (O, LSE) is merged into the
-query chunk's running result.  While step s computes, the shard for step
+pair is one fa_fwd_merge call on (C x C) chunks, which folds the pair's
+(O, LSE) into the query chunk's running fp32 result in its epilogue.  While step s computes, the shard for step
 s+1 is already travelling: each rank sends what it holds to rank r+1 and
 receives from rank r-1 (NCCL send/recv over NVLink on GPUs, gloo on CPU).
 
-Backward on rank r.  The same pairs, each one fa_bwd call given the query
-chunk's FULL output and LSE (so every pair's dQ, dK, dV are exact terms of the
-whole-sequence gradient).  dQ terms are summed locally in fp32; the fp32
-dK/dV sums of a K/V shard travel with it around the ring and, after R hops,
-reach their owner complete.  The next step's K/V transfer overlaps the current
-step's kernels; a step's pair gradients are computed before the incoming dK/dV
-sums are waited for.
+Backward on rank r.  The same pairs, each against the query chunk's FULL
+output and LSE (so every pair's dQ, dK, dV are exact terms of the
+whole-sequence gradient): the row statistics of each query chunk are formed
+once (fa_bwd_stats), and every pair is one fa_bwd_accumulate call that adds
+its dQ into the chunk's local fp32 sum and its dK, dV into the fp32 sums of
+the K/V shard it holds.  Those sums travel with the shard around the ring and,
+after R hops, reach their owner complete.  The next step's K/V transfer
+overlaps the current step's kernels; the incoming dK/dV sums are waited for
+before the step's pairs add into them.
 
 The per-pair arithmetic, the merge and the accumulation run in the sm_100a
 kernels of the C ABI (KernelOps); this module only plans the pairs and moves
@@ -135,6 +137,17 @@ class KernelOps:
     def merge(self, o_acc, lse_acc, o_part, lse_part, first: bool, out=None):
         self.A.lse_merge(o_acc, lse_acc, o_part, lse_part, first=first, out=out)
 
+    def fwd_merge(self, q, k, v, causal_flag: bool, scale: float, o_acc, lse_acc, first: bool, out=None):
+        self.A.fwd_merge(q, k, v, o_acc, lse_acc, causal=causal_flag, scale=scale, first=first, out=out)
+
+    def bwd_prepare(self, o, do, lse, scale: float):
+        return self.A.bwd_stats(o, do, lse, scale=scale)
+
+    def bwd_accumulate(self, q, k, v, do, prep, causal_flag: bool, scale: float, dq_acc, dk_acc, dv_acc,
+                       first_dq: bool, first_dkv: bool):
+        self.A.bwd_accumulate(q, k, v, do, prep, dq_acc, dk_acc, dv_acc, causal=causal_flag, scale=scale,
+                              first_dq=first_dq, first_dkv=first_dkv)
+
     def accumulate(self, acc, src, first: bool, out=None):
         self.A.accumulate(acc, src, first=first, out=out)
 
@@ -171,42 +184,38 @@ class _FwdRank:
 
     def step(self, s, k_cur, v_cur):
         for i, (qs, ks, cflag) in enumerate(self.plans[s][1]):
-            o_p, lse_p = self.ops.fwd(self.q[qs], k_cur[ks], v_cur[ks], cflag, self.scale)
-            self.ops.merge(self.o_acc[qs], self.lse[qs], o_p, lse_p, first=not self.started[qs],
-                           out=self.out[qs] if self.last[qs] == (s, i) else None)
+            self.ops.fwd_merge(self.q[qs], k_cur[ks], v_cur[ks], cflag, self.scale, self.o_acc[qs], self.lse[qs],
+                               first=not self.started[qs], out=self.out[qs] if self.last[qs] == (s, i) else None)
             self.started[qs] = True
 
 
 class _BwdRank:
-    """One rank's backward: local fp32 dQ sums, pair gradients for the
-    travelling dK/dV sums."""
+    """One rank's backward: row statistics once per query chunk, local fp32
+    dQ sums, pair gradients added straight into the travelling dK/dV sums."""
 
     def __init__(self, ops, rank, world, q, o, do, lse, causal, scale):
-        self.ops, self.q, self.o, self.do, self.scale = ops, q, o, do, scale
-        self.lse = [lse[0], lse[1]]   # fa_bwd reads LSE one element at a time (4-byte alignment)
+        self.ops, self.q, self.do, self.scale = ops, q, do, scale
+        # fa_bwd_stats reads LSE one element at a time (4-byte alignment)
+        self.prep = [ops.bwd_prepare(o[i], do[i], lse[i], scale) for i in (0, 1)]
         self.plans = ring_plans(rank, world, causal)
         self.last = _last_use(self.plans)
         self.dq_acc = ops.empty_acc(q.shape, q)
         self.dq = torch.empty_like(q)
         self.started = [False, False]
 
-    def partials(self, s, k_cur, v_cur):
-        return [(qs, ks, self.ops.bwd(self.q[qs], k_cur[ks], v_cur[ks], self.o[qs], self.do[qs], self.lse[qs],
-                                      cflag, self.scale))
-                for qs, ks, cflag in self.plans[s][1]]
-
-    def absorb(self, s, parts, dk_acc, dv_acc):
-        """Add step s's pair gradients: dQ locally, dK/dV into the sums of the
+    def step(self, s, k_cur, v_cur, dk_acc, dv_acc):
+        """Step s's pairs: dQ into the local sums, dK/dV into the sums of the
         shard this rank holds (fresh at step 0, when the shard is its own)."""
         touched = [False, False]
-        for i, (qs, ks, (dq_p, dk_p, dv_p)) in enumerate(parts):
-            self.ops.accumulate(self.dq_acc[qs], dq_p, first=not self.started[qs],
-                                out=self.dq[qs] if self.last[qs] == (s, i) else None)
-            self.started[qs] = True
+        for i, (qs, ks, cflag) in enumerate(self.plans[s][1]):
             fresh = s == 0 and not touched[ks]
-            self.ops.accumulate(dk_acc[ks], dk_p, first=fresh)
-            self.ops.accumulate(dv_acc[ks], dv_p, first=fresh)
+            self.ops.bwd_accumulate(self.q[qs], k_cur[ks], v_cur[ks], self.do[qs], self.prep[qs], cflag, self.scale,
+                                    self.dq_acc[qs], dk_acc[ks], dv_acc[ks], first_dq=not self.started[qs],
+                                    first_dkv=fresh)
+            self.started[qs] = True
             touched[ks] = True
+            if self.last[qs] == (s, i):
+                self.ops.accumulate(self.dq_acc[qs], None, first=False, out=self.dq[qs])
         if s == 0:
             for ks in (0, 1):
                 if not touched[ks]:
@@ -252,7 +261,7 @@ def virtual_ring_bwd(q_shards, k_shards, v_shards, o_shards, do_shards, lse_shar
     for s in range(R):
         for r in range(R):
             src = (r - s) % R
-            ranks[r].absorb(s, ranks[r].partials(s, k_shards[src], v_shards[src]), dk_acc[src], dv_acc[src])
+            ranks[r].step(s, k_shards[src], v_shards[src], dk_acc[src], dv_acc[src])
     out = []
     for r in range(R):
         dk, dv = torch.empty_like(k_shards[r]), torch.empty_like(v_shards[r])
@@ -331,11 +340,10 @@ def ring_attention_bwd(q, k, v, o, do, lse, causal: bool = True, scale: float | 
     acc_works = None
     for s in range(R):
         kv_works = comm.shift(cur, kv_bufs[s % 2]) if s + 1 < R else None
-        parts = me.partials(s, *cur)
         if acc_works is not None:
             _wait(acc_works)
             acc_cur = acc[s % 2]
-        me.absorb(s, parts, *acc_cur)
+        me.step(s, *cur, *acc_cur)
         if R > 1:
             # the sums move on every step, the last hop bringing them home
             acc_works = comm.shift(acc_cur, acc[(s + 1) % 2])

@@ -325,14 +325,33 @@ const char* fa_status_str(fa_status s) {
     return "unknown status";
 }
 
-fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
-                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Forward of fa_fwd (merge == nullptr) and fa_fwd_merge.
+struct MergeArgs {
+    float* o_acc;
+    float* lse_acc;
+    void* o_out;
+    int first;
+};
+
+fa_status fwd_impl(const fa_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
+                   const MergeArgs* merge, void* stream) {
     fa_status st = check_shape(shape);
     if (st != FA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v)) return FA_ERR_INVALID_ARG;
+    if (merge) {
+        if (!aligned16(merge->o_acc) || !aligned4(merge->lse_acc) ||
+            (merge->o_out != nullptr && !aligned16(merge->o_out)))
+            return FA_ERR_INVALID_ARG;
+    } else if (!aligned16(o) || !aligned16(lse)) {
+        return FA_ERR_INVALID_ARG;
+    }
     if ((st = check_device()) != FA_OK) return st;
     const fa_shape& s = *shape;
-    const bool pair = fwd_use_pair(s);
+    const bool pair = !merge && fwd_use_pair(s);   // the merge epilogue lives in the one-CTA kernel
     CUtensorMap tq, tk, tv;
     if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D, 2, pair ? kTileN / 2 : kTileN) ||
         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D))
@@ -355,12 +374,31 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void
     p.o = o;
     p.lse = lse;
     p.o_scale = 1.f;
+    p.m_o = merge ? merge->o_acc : nullptr;
+    p.m_lse = merge ? merge->lse_acc : nullptr;
+    p.m_out = merge ? merge->o_out : nullptr;
+    p.m_first = merge ? (merge->first ? 1 : 0) : 0;
     p.n_units = p.n_mblocks * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     if ((st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
     cudaError_t e = pair ? timed(10, strm, [&] { return launch_fwd_pair(tq, tk, tv, p, strm); })
                          : timed(0, strm, [&] { return launch_fwd(s.D, tq, tk, tv, p, strm); });
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k, const void* v, void* o, float* lse,
+                 void* stream) {
+    return fwd_impl(shape, q, k, v, o, lse, nullptr, stream);
+}
+
+fa_status fa_fwd_merge(const fa_shape* shape, const void* q, const void* k, const void* v, float* o_acc,
+                       float* lse_acc, void* o_out, int first, void* stream) {
+    const MergeArgs m{o_acc, lse_acc, o_out, first};
+    return fwd_impl(shape, q, k, v, nullptr, nullptr, &m, stream);
 }
 
 fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const void* v, float q_scale,
@@ -394,6 +432,10 @@ fa_status fa_fwd_fp8(const fa_shape* shape, const void* q, const void* k, const 
     p.o = o;
     p.lse = lse;
     p.o_scale = v_scale;
+    p.m_o = nullptr;
+    p.m_lse = nullptr;
+    p.m_out = nullptr;
+    p.m_first = 0;
     p.n_units = p.n_mblocks * s.B * s.Hq;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
     if ((st = fwd_sched_slot(strm, &p.sched)) != FA_OK) return st;
@@ -443,26 +485,47 @@ size_t fa_bwd_workspace_bytes(const fa_shape* shape) {
     return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total;
 }
 
-fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v, const void* o, const void* dout,
-                 const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// What bwd_impl runs: the whole backward (fa_bwd), only the row statistics
+// into the workspace (fa_bwd_stats), or the two passes on statistics already
+// in the workspace, adding into fp32 sums (fa_bwd_accumulate).
+enum BwdMode { kBwdFull, kBwdStats, kBwdAccumulate };
+struct AccArgs {
+    float* dq;
+    float* dk;
+    float* dv;
+    int first_dq, first_dkv;
+};
+
+fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const void* k, const void* v, const void* o,
+                   const void* dout, const float* lse, void* dq, void* dk, void* dv, const AccArgs* acc,
+                   void* workspace, size_t workspace_bytes, void* stream) {
     fa_status st = check_shape(shape);
     if (st != FA_OK) return st;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned4(lse) ||
-        !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    const bool need_stats_in = mode != kBwdAccumulate;
+    const bool need_passes = mode != kBwdStats;
+    if (need_stats_in && (!aligned16(o) || !aligned16(dout) || !aligned4(lse))) return FA_ERR_INVALID_ARG;
+    if (need_passes && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout))) return FA_ERR_INVALID_ARG;
+    if (mode == kBwdFull && (!aligned16(dq) || !aligned16(dk) || !aligned16(dv))) return FA_ERR_INVALID_ARG;
+    if (mode == kBwdAccumulate && (!acc || !aligned16(acc->dq) || !aligned16(acc->dk) || !aligned16(acc->dv)))
         return FA_ERR_INVALID_ARG;
     const fa_shape& s = *shape;
-    const bool separate = dq_separate_mode();
+    // the statistics entry points always use the separate passes' layout
+    const bool separate = mode != kBwdFull || dq_separate_mode();
     const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D, !separate);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws.total)
         return FA_ERR_INVALID_ARG;
     if ((st = check_device()) != FA_OK) return st;
     CUtensorMap tq, tk, tv, tdo;
-    if (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
-        !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D))
+    if (need_passes && (!make_map(&tq, q, s.B * s.Hq, s.N, s.D) || !make_map(&tk, k, s.B * s.Hkv, s.N, s.D) ||
+                        !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D)))
         return FA_ERR_CUDA;
-    const bool pair_dkdv = separate && bwd_dkdv_use_pair(s);
-    const bool pair_dq = separate && bwd_dq_use_pair(s);
+    // the accumulate epilogues live in the one-CTA passes
+    const bool pair_dkdv = mode == kBwdFull && separate && bwd_dkdv_use_pair(s);
+    const bool pair_dq = mode == kBwdFull && separate && bwd_dq_use_pair(s);
     CUtensorMap tq_half, tdo_half, tk_half, tv_half;
     if (pair_dkdv && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
                       !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2)))
@@ -507,13 +570,25 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
     p.sched = reinterpret_cast<unsigned int*>(wsb + ws.sched_off);
     p.n_units_dkdv = (pair_dkdv ? (s.N + 2 * kTileN - 1) / (2 * kTileN) : T) * s.B * s.Hkv;
     p.n_units_dq = (pair_dq ? (s.N + 2 * kTileM - 1) / (2 * kTileM) : T) * s.B * s.Hq;
+    p.a_dq = mode == kBwdAccumulate ? acc->dq : nullptr;
+    p.a_dk = mode == kBwdAccumulate ? acc->dk : nullptr;
+    p.a_dv = mode == kBwdAccumulate ? acc->dv : nullptr;
+    p.a_first_dq = mode == kBwdAccumulate && acc->first_dq ? 1 : 0;
+    p.a_first_dkv = mode == kBwdAccumulate && acc->first_dkv ? 1 : 0;
     cudaStream_t strm = static_cast<cudaStream_t>(stream);
-    cudaError_t e = timed(1, strm, [&] {
-        return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
-                                     reinterpret_cast<float*>(wsb + ws.dvec_off), separate ? nullptr : p.dq_acc,
-                                     s.B * s.Hq, s.N, Npad, s.scale,
-                                     reinterpret_cast<unsigned int*>(wsb + ws.sched_off), strm);
-    });
+    cudaError_t e = cudaSuccess;
+    if (need_stats_in) {
+        e = timed(1, strm, [&] {
+            return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
+                                         reinterpret_cast<float*>(wsb + ws.dvec_off), separate ? nullptr : p.dq_acc,
+                                         s.B * s.Hq, s.N, Npad, s.scale,
+                                         reinterpret_cast<unsigned int*>(wsb + ws.sched_off), strm);
+        });
+    } else {
+        // statistics already in the workspace; only the work counters restart
+        e = cudaMemsetAsync(wsb + ws.sched_off, 0, kSchedCounters * sizeof(unsigned int), strm);
+    }
+    if (!need_passes) return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
     if (separate) {
         if (e == cudaSuccess)
             e = pair_dkdv ? timed(11, strm, [&] { return launch_bwd_dkdv_pair(tq, tq_half, tk, tv, tdo, tdo_half, p, strm); })
@@ -529,6 +604,31 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void
             });
     }
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    return bwd_impl(kBwdFull, shape, q, k, v, o, dout, lse, dq, dk, dv, nullptr, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_stats(const fa_shape* shape, const void* o, const void* dout, const float* lse, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    return bwd_impl(kBwdStats, shape, nullptr, nullptr, nullptr, o, dout, lse, nullptr, nullptr, nullptr, nullptr,
+                    workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_accumulate(const fa_shape* shape, const void* q, const void* k, const void* v, const void* dout,
+                            float* dq_acc, float* dk_acc, float* dv_acc, int flags, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    if (flags & ~(FA_ACC_DQ_FIRST | FA_ACC_DKV_FIRST)) return FA_ERR_INVALID_ARG;
+    const AccArgs a{dq_acc, dk_acc, dv_acc, (flags & FA_ACC_DQ_FIRST) ? 1 : 0, (flags & FA_ACC_DKV_FIRST) ? 1 : 0};
+    return bwd_impl(kBwdAccumulate, shape, q, k, v, nullptr, dout, nullptr, nullptr, nullptr, nullptr, &a, workspace,
+                    workspace_bytes, stream);
 }
 
 // fa_bwd with its workspace taken from the library's static scratch instead of

@@ -62,6 +62,21 @@ __host__ __device__ constexpr uint32_t packed_col(int kk) {
     return static_cast<uint32_t>((kk / (kCols / 16)) * kCols + (kk % (kCols / 16)) * 8);
 }
 
+// acc[0..15] = (first ? 0 : acc[0..15]) + the 16 fp32 values in v (one
+// thread's row segment; 16-byte accesses).
+__device__ __forceinline__ void accumulate16(float* acc, const uint32_t (&v)[16], int first) {
+    float4* a4 = reinterpret_cast<float4*>(acc);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float4 a = first ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[t];
+        a.x += __uint_as_float(v[4 * t]);
+        a.y += __uint_as_float(v[4 * t + 1]);
+        a.z += __uint_as_float(v[4 * t + 2]);
+        a.w += __uint_as_float(v[4 * t + 3]);
+        a4[t] = a;
+    }
+}
+
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int site) {
     if (mbar_try_wait(bar, parity)) return;
     unsigned long long t0 = globaltimer_ns();
@@ -481,11 +496,16 @@ fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
                 __nv_bfloat16* dst_row =
                     reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * D + wg * kPer;
+                float* acc_row = p.a_dk ? (which == 0 ? p.a_dv : p.a_dk) + row * D + wg * kPer : nullptr;
 #pragma unroll 1
                 for (int q = 0; q < kPer / 16; ++q) {
                     uint32_t v16[16];
                     tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
                     tmem_ld_wait();
+                    if (acc_row) {   // accumulate mode: fp32 sums instead of bf16 outputs
+                        if (kv_ok) accumulate16(acc_row + q * 16, v16, p.a_first_dkv);
+                        continue;
+                    }
                     uint32_t pk[8];
 #pragma unroll
                     for (int t = 0; t < 8; ++t)
@@ -835,11 +855,16 @@ fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             constexpr int kPer = D / kGroups;   // head-dimension columns written by this group
             __nv_bfloat16* dst_row =
                 reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(w.bh) * p.N + qrow) * D + wg * kPer;
+            float* acc_row = p.a_dq ? p.a_dq + (static_cast<size_t>(w.bh) * p.N + qrow) * D + wg * kPer : nullptr;
 #pragma unroll 1
             for (int q = 0; q < kPer / 16; ++q) {
                 uint32_t v16[16];
                 tmem_ld16(tmem + lane_off + kColDQ + wg * kPer + q * 16, v16);
                 tmem_ld_wait();
+                if (acc_row) {   // accumulate mode: fp32 sums instead of bf16 outputs
+                    if (qrow < p.N) accumulate16(acc_row + q * 16, v16, p.a_first_dq);
+                    continue;
+                }
                 uint32_t pk[8];
 #pragma unroll
                 for (int t = 0; t < 8; ++t)

@@ -70,6 +70,60 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
     }
 }
 
+// Merge-mode epilogue of one query row (thread = row): this call's result
+// over its keys, O / l with LSE_p = ln 2 (m + log2 l), is folded into the
+// running fp32 result of the row by the log-sum-exp rule,
+//   LSE = log(e^LSE_old + e^LSE_p),  O = e^(LSE_old - LSE) O_old + e^(LSE_p - LSE) O / l,
+// or replaces it when p.m_first is set ("【词汇专栏】FlashAttention：大模型训练的
+// 加速器", section 3.2 item 2: the exact join of sequence parts).
+template <int D>
+__device__ __forceinline__ void merge_epilogue(const FwdParams& p, uint32_t tO, size_t row, bool valid, float m_used,
+                                               float l) {
+    constexpr float kLog2e = 1.4426950408889634f;
+    constexpr float kLn2 = 0.69314718055994531f;
+    const float lse_p = (m_used + lg2(l)) * kLn2;
+    float w_old = 0.f, w_new = 1.f, lse_n = lse_p;
+    if (!p.m_first && valid) {
+        const float lse_o = p.m_lse[row];
+        const float mx = fmaxf(lse_o, lse_p);
+        const float eo = ex2((lse_o - mx) * kLog2e);   // 0 when lse_o = -inf (no keys so far)
+        const float ep = ex2((lse_p - mx) * kLog2e);
+        const float inv = 1.f / (eo + ep);
+        w_old = eo * inv;
+        w_new = ep * inv;
+        lse_n = mx + lg2(eo + ep) * kLn2;
+    }
+    const float wn = w_new / l;
+    float* oacc = p.m_o + row * D;
+    __nv_bfloat16* oout = p.m_out ? reinterpret_cast<__nv_bfloat16*>(p.m_out) + row * D : nullptr;
+#pragma unroll 1
+    for (int q = 0; q < D / 32; ++q) {
+        uint32_t ov[32];
+        tmem_ld32(tO + q * 32, ov);
+        tmem_ld_wait();
+        if (!valid) continue;
+        float4* a4 = reinterpret_cast<float4*>(oacc + q * 32);
+        uint32_t pk[16];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            float4 a = p.m_first ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[t];
+            a.x = fmaf(w_old, a.x, wn * __uint_as_float(ov[4 * t]));
+            a.y = fmaf(w_old, a.y, wn * __uint_as_float(ov[4 * t + 1]));
+            a.z = fmaf(w_old, a.z, wn * __uint_as_float(ov[4 * t + 2]));
+            a.w = fmaf(w_old, a.w, wn * __uint_as_float(ov[4 * t + 3]));
+            a4[t] = a;
+            pk[2 * t] = pack_bf16x2(a.x, a.y);
+            pk[2 * t + 1] = pack_bf16x2(a.z, a.w);
+        }
+        if (oout) {
+            uint4* dst = reinterpret_cast<uint4*>(oout + q * 32);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) dst[t] = make_uint4(pk[4 * t], pk[4 * t + 1], pk[4 * t + 2], pk[4 * t + 3]);
+        }
+    }
+    if (valid) p.m_lse[row] = lse_n;
+}
+
 // One forward work unit: (batch x head bh, pair of 128-row query tiles mb).
 // Units are numbered head group by head group, heaviest (last) query block
 // first inside a group, then head.
@@ -421,6 +475,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             tc_fence_after();
             const float inv_l = 1.f / l;
             const bool valid = qrow < p.N;
+            if (p.m_o != nullptr) {
+                merge_epilogue<D>(p, tO, static_cast<size_t>(w.bh) * p.N + qrow, valid, m_used, l);
+                tc_fence_before();
+                continue;
+            }
             __nv_bfloat16* orow_g =
                 reinterpret_cast<__nv_bfloat16*>(p.o) + (static_cast<size_t>(w.bh) * p.N + qrow) * D;
 #pragma unroll 1

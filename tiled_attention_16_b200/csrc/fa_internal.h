@@ -26,6 +26,14 @@ struct FwdParams {
     float o_scale;     // multiplies O before the 1/l normalisation (FP8: V's descale; 1 for bf16)
     int n_units;       // work units: B * Hq * n_mblocks
     unsigned int* sched;  // [2] counter slot of the persistent forward: next unit, CTAs done
+    // Merge mode (one-CTA kernel only; m_o == nullptr: off): instead of writing
+    // o and lse, fold this call's result into a running fp32 result by the
+    // log-sum-exp rule; m_first: set it from this call.  m_out (bf16, may be
+    // null) also receives the merged rows.
+    float* m_o;        // fp32 [B,Hq,N,D]
+    float* m_lse;      // fp32 [B,Hq,N]
+    void* m_out;
+    int m_first;
 };
 
 // Multiprocessor count of the current device (cached per device; -1 on error).
@@ -47,6 +55,13 @@ struct BwdParams {
     unsigned int* sched;     // work counters of the persistent kernels (zeroed by the preprocess)
     int n_units_dkdv;        // work units of the dK/dV pass
     int n_units_dq;          // work units of the dQ pass
+    // Accumulate mode of the one-CTA separate passes (nullptr: off): add the
+    // gradients into fp32 buffers instead of writing dq / dk / dv; the first
+    // flags overwrite instead of adding.
+    float* a_dq;       // fp32 [B,Hq,N,D]
+    float* a_dk;       // fp32 [B,Hkv,N,D]
+    float* a_dv;       // fp32 [B,Hkv,N,D]
+    int a_first_dq, a_first_dkv;
 };
 
 // Counters at the start of the backward workspace: [0] dK/dV pass, [1] dQ pass.
