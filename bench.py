@@ -120,6 +120,7 @@ KERNEL_FILES = {
     "fa_bwd_dq_pair_kernel": ("fa_bwd_pair.cu", "fa_bwd.cu"),
     "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_kernel": ("fa_bwd.cu",),
+    "fa_bwd_preprocess": ("fa_bwd.cu",),
     "fa_decode_split_kernel": ("fa_decode.cu",),
     "fa_decode_combine_kernel": ("fa_decode.cu",),
 }
