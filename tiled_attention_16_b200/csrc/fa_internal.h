@@ -34,6 +34,7 @@ struct FwdParams {
     float* m_lse;      // fp32 [B,Hq,N]
     void* m_out;
     int m_first;
+    int fma_exp;       // one-CTA bf16 kernel: 1/8 of the exponentials on the FMA pipe
 };
 
 // Multiprocessor count of the current device (cached per device; -1 on error).
