@@ -120,6 +120,7 @@ KERNEL_FILES = {
     "fa_bwd_dq_pair_kernel": ("fa_bwd_pair.cu", "fa_bwd.cu"),
     "fa_bwd_dq_kernel": ("fa_bwd_split.cu", "fa_bwd.cu"),
     "fa_bwd_kernel": ("fa_bwd.cu",),
+    "fa_bwd_fused_kernel": ("fa_bwd_fused.cu", "fa_bwd.cu"),
     "fa_bwd_preprocess": ("fa_bwd.cu",),
     "fa_decode_split_kernel": ("fa_decode.cu",),
     "fa_decode_combine_kernel": ("fa_decode.cu",),
@@ -326,6 +327,7 @@ def run_gpu(args, wl):
     # dQ kernel 3 (S and dP recomputed, dQ).
     gemm = wl.flops_fwd() / 2
     kernel_flops = {"fa_fwd_kernel": 2 * gemm, "fa_fwd_pair_kernel": 2 * gemm, "fa_bwd_kernel": 5 * gemm,
+                    "fa_bwd_fused_kernel": 5 * gemm,
                     "fa_bwd_dkdv_kernel": 4 * gemm, "fa_bwd_dkdv_pair_kernel": 4 * gemm, "fa_bwd_dq_kernel": 3 * gemm,
                     "fa_bwd_dq_pair_kernel": 3 * gemm}
     tensor_k = {k: v for k, v in kms.items() if v and k in kernel_flops}
@@ -339,7 +341,7 @@ def run_gpu(args, wl):
                 "flops_per_launch": kernel_flops[dominant]}
     fwd_tf = wl.flops_fwd() / (fwd_ms * 1e-3) / 1e12
     bwd_tf = wl.flops_bwd() / (bwd_ms * 1e-3) / 1e12
-    pre_zero = wl.B * wl.Hq * wl.N * wl.D * 4 if kms.get("fa_bwd_kernel") else 0
+    pre_zero = wl.B * wl.Hq * wl.N * wl.D * 4 if (kms.get("fa_bwd_kernel") or kms.get("fa_bwd_fused_kernel")) else 0
     pre_bytes = wl.B * wl.Hq * wl.N * (2 * wl.D * 2 + 4 + 8) + pre_zero
     conv_bytes = wl.B * wl.Hq * wl.N * wl.D * (4 + 2)
     breakdown = {

@@ -124,12 +124,36 @@ FA_API size_t fa_decode_workspace_bytes(const fa_kv_shape* shape);
 FA_API fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* k, const void* v, void* o,
                     float* lse, void* workspace, size_t workspace_bytes, void* stream);
 
-/* Bytes of device workspace fa_bwd needs for `shape` (0 if the shape is invalid):
- * two work counters and the per-row statistics (LSE in log2 units and
- * D = rowsum(dO o O), each padded to a multiple of 128 rows), about
- * 8 * B * Hq * N bytes; plus an fp32 dQ accumulator [B,Hq,N,D] when the
- * environment variable FA_DQ_MODE=atomic selects the fused backward (the
- * mode is read once per process, so the size is stable within a process). */
+/* How fa_bwd forms dQ ("FlashAttention V2深度解析：反向传播显存优化让大模型训练
+ * 不再OOM", section 改进2 parallelises the key sequence, so several key blocks
+ * contribute to each dQ row):
+ *   FA_BWD_FUSED          one persistent kernel runs all five GEMMs per tile
+ *                         pair; each key block's dQ partial is added into an
+ *                         fp32 accumulator by reductions in L2, in an order
+ *                         that varies from run to run (dK, dV do not vary).
+ *   FA_BWD_DETERMINISTIC  a dK/dV pass and a separate dQ pass that recomputes
+ *                         S and dP (seven GEMMs per tile pair, no reductions);
+ *                         repeated calls are bitwise equal.
+ *   FA_BWD_AUTO           (default) the measured choice: FA_BWD_FUSED for
+ *                         D = 128 (10-11% faster at N = 8192 and 65536, equal
+ *                         at N = 2048), FA_BWD_DETERMINISTIC for D = 64.
+ * fa_set_bwd_mode sets the process-wide choice (FA_ERR_INVALID_ARG for other
+ * values) and fa_get_bwd_mode returns it; neither touches the GPU.  The
+ * environment variable FA_DQ_MODE=separate|fused (read once per process)
+ * overrides both.  Set the mode before querying fa_bwd_workspace_bytes: the
+ * fused mode needs the larger workspace.  Calls already enqueued are not
+ * affected by a later change. */
+#define FA_BWD_AUTO 0
+#define FA_BWD_DETERMINISTIC 1
+#define FA_BWD_FUSED 2
+FA_API fa_status fa_set_bwd_mode(int mode);
+FA_API int fa_get_bwd_mode(void);
+
+/* Bytes of device workspace fa_bwd needs for `shape` under the current
+ * backward mode (0 if the shape is invalid): two work counters and the
+ * per-row statistics (LSE in log2 units and D = rowsum(dO o O), each padded
+ * to a multiple of 128 rows), about 8 * B * Hq * N bytes; plus an fp32 dQ
+ * accumulator [B,Hq,N,D] when the shape runs the fused backward. */
 FA_API size_t fa_bwd_workspace_bytes(const fa_shape* shape);
 
 /* Backward.  Inputs q, k, v, o, dout (bf16) and lse (fp32, as written by
@@ -144,9 +168,10 @@ FA_API fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k, con
 /* Backward that allocates nothing (the pages have no counterpart: this is a
  * deployment convenience, not part of the method).
  *
- * Same computation, arguments and outputs as fa_bwd, but without a caller
- * workspace: the scratch it needs (the per-row LSE/D statistics and the fp32
- * dQ accumulator of the fused mode, fa_bwd_workspace_bytes(shape) bytes) lives in a fixed
+ * Same computation, arguments and outputs as fa_bwd in FA_BWD_DETERMINISTIC
+ * mode (whatever the current mode: bitwise equal to it), but without a caller
+ * workspace: the scratch it needs (the work counters and the per-row LSE/D
+ * statistics, about 8 * B * Hq * N bytes) lives in a fixed
  * FA_NOALLOC_SCRATCH_BYTES region of device memory that the library reserves
  * statically on every GPU that loads it, held until the process exits.  It is
  * meant for callers that cannot call cudaMalloc or hand out device memory on
@@ -228,9 +253,11 @@ FA_API fa_status fa_fwd_merge(const fa_shape* shape, const void* q, const void* 
  *          FA_ACC_DKV_FIRST: the same for dk_acc and dv_acc.
  * The workspace must hold the statistics fa_bwd_stats wrote for the same
  * shape and the same o, dout and lse; its work counters are reset here.  q,
- * k, v, dout as for fa_bwd (dout is read again by the passes).  Always the
- * one-CTA passes with the separate dQ pass (whatever FA_BWD_TILE and
- * FA_DQ_MODE say).  Errors and asynchrony as for fa_bwd. */
+ * k, v, dout as for fa_bwd (dout is read again by the passes).  For D = 128
+ * in the fused backward mode (the default) one fused kernel runs and its
+ * fp32 reductions add each dQ term straight into dq_acc (cleared first by a
+ * FA_ACC_DQ_FIRST call), so dq_acc sums in varying order; otherwise the
+ * one-CTA separate passes run (whatever FA_BWD_TILE says).  Errors and asynchrony as for fa_bwd. */
 #define FA_ACC_DQ_FIRST 1
 #define FA_ACC_DKV_FIRST 2
 FA_API fa_status fa_bwd_stats(const fa_shape* shape, const void* o, const void* dout, const float* lse,
@@ -281,13 +308,15 @@ FA_API unsigned int fa_debug_timeout_sites(void);
  * kernel, 6 FP8 forward, 7 decode (split kernel and combine together),
  * 8 log-sum-exp merge, 9 accumulation, 10 forward on CTA pairs (256-row MMA
  * tiles), 11 backward dK/dV kernel on CTA pairs (256-key blocks), 12
- * backward dQ kernel on CTA pairs (256-query blocks) (FA_PROFILE_KINDS;
- * fa_fwd uses 0, or 10 when the environment variable FA_FWD_TILE=m256 selects
- * the CTA-pair kernel for D = 128; fa_bwd uses 1, 4, 5 by default,
- * FA_BWD_TILE=m256 selects the CTA-pair passes (1, 11, 12) for D = 128, and
- * FA_DQ_MODE=atomic the fused kernel (1, 2, 3)).  Events are host-created objects; no device
+ * backward dQ kernel on CTA pairs (256-query blocks), 13 persistent fused
+ * backward for D = 128 (dK, dV and dQ by fp32 bulk reductions)
+ * (FA_PROFILE_KINDS; fa_fwd uses 0, or 10 when the environment variable
+ * FA_FWD_TILE=m256 selects the CTA-pair kernel for D = 128; fa_bwd uses 1,
+ * 13, 3 in the fused mode for D = 128 (1, 2, 3 for D = 64) and 1, 4, 5 in
+ * the deterministic mode, where FA_BWD_TILE=m256 selects the CTA-pair passes
+ * (1, 11, 12) for D = 128).  Events are host-created objects; no device
  * memory is allocated. */
-#define FA_PROFILE_KINDS 13
+#define FA_PROFILE_KINDS 14
 FA_API fa_status fa_profile_begin(void);
 FA_API fa_status fa_profile_end(float* total_ms, int* launches);
 

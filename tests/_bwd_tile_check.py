@@ -42,6 +42,7 @@ def main() -> int:
     expect = {"m256": {"fa_bwd_dkdv_pair_kernel", "fa_bwd_dq_pair_kernel"},
               "m128": {"fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel"}}[tile]
     dev = torch.device("cuda:0")
+    A.set_bwd_mode("deterministic")   # the tile variants are those of the separate passes
     for (B, Hq, Hkv, N, causal, sqk) in CASES:
         wl = Workload("btile", B=B, Hq=Hq, Hkv=Hkv, N=N, D=128, causal=causal, seed=900 + N + Hq, sigma_qk=sqk)
         q, k, v, do = make_inputs(wl)

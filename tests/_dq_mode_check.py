@@ -23,8 +23,7 @@ CASES = [(1, 2, 2, 128, 64, False), (2, 3, 3, 17, 128, True), (1, 4, 2, 300, 128
 
 
 def main() -> int:
-    mode = os.environ.get("FA_DQ_MODE", "separate")
-    expect = {"fa_bwd_kernel", "fa_bwd_dq_convert"} if mode == "atomic" else {"fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel"}
+    mode = os.environ.get("FA_DQ_MODE", "auto")
     dev = torch.device("cuda:0")
     for (B, Hq, Hkv, N, D, causal) in CASES:
         wl = Workload("mode", B=B, Hq=Hq, Hkv=Hkv, N=N, D=D, causal=causal, seed=500 + N + D)
@@ -32,6 +31,9 @@ def main() -> int:
         sc = wl.softmax_scale
         qd, kd, vd, dod = (x.to(dev) for x in (q, k, v, do))
         o, lse = A.fwd(qd, kd, vd, causal=causal, scale=sc)
+        fused = mode in ("atomic", "fused") or (mode == "auto" and D == 128)   # auto: fused for D = 128
+        expect = ({"fa_bwd_fused_kernel" if D == 128 else "fa_bwd_kernel", "fa_bwd_dq_convert"} if fused
+                  else {"fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel"})
         A.profile_begin()
         grads = A.bwd(qd, kd, vd, o, dod, lse, causal=causal, scale=sc)
         ran = {name for name, (_, n) in A.profile_end().items() if n}

@@ -48,7 +48,7 @@ int main(void) {
     CHECK(15, fa_accumulate(0, NULL, NULL, NULL, 1, NULL) == FA_OK);
     CHECK(16, strcmp(fa_status_str(FA_OK), "ok") == 0 && fa_status_str((fa_status)99) != NULL);
     CHECK(17, fa_debug_timeout_sites() == 0u);
-    CHECK(18, FA_PROFILE_KINDS == 13 && FA_NOALLOC_SCRATCH_BYTES == (32u << 20));
+    CHECK(18, FA_PROFILE_KINDS == 14 && FA_NOALLOC_SCRATCH_BYTES == (32u << 20));
     CHECK(19, fa_selftest_wait_timeout(3, 3, NULL) == FA_ERR_INVALID_ARG);
     printf("c abi ok\n");
     return 0;

@@ -22,7 +22,7 @@ def test_exports_every_declared_symbol():
                           "fa_status_str", "fa_debug_timeout_sites", "fa_profile_begin", "fa_profile_end",
                           "fa_bwd_noalloc", "fa_fwd_fp8", "fa_decode", "fa_decode_workspace_bytes",
                           "fa_lse_merge", "fa_accumulate", "fa_selftest_wait_timeout", "fa_fwd_merge",
-                          "fa_bwd_stats", "fa_bwd_accumulate"}
+                          "fa_bwd_stats", "fa_bwd_accumulate", "fa_set_bwd_mode", "fa_get_bwd_mode"}
     L = A.lib()
     for n in names:
         assert hasattr(L, n), n
@@ -117,8 +117,9 @@ def test_workspace_bytes_formula():
         s = A.make_shape(B, Hq, 1, N, D, 0.1, 0)
         npad = -(-N // 128) * 128
         up = lambda x: -(-x // 256) * 256  # noqa: E731
-        # counters, lse2, D; the fp32 dQ accumulator only for the fused (atomic) mode
-        fused = os.environ.get("FA_DQ_MODE") == "atomic"
+        # counters, lse2, D; the fp32 dQ accumulator only for the fused mode (default for D = 128)
+        env = os.environ.get("FA_DQ_MODE")
+        fused = env in ("atomic", "fused") or (env != "separate" and D == 128)
         expect = up(4 * 4) + 2 * up(B * Hq * npad * 4) + (up(B * Hq * N * D * 4) if fused else 0)
         assert A.lib().fa_bwd_workspace_bytes(ctypes.byref(s)) == expect
 
@@ -142,7 +143,7 @@ def test_profile_hooks_without_launches():
     A.profile_begin()
     res = A.profile_end()
     assert set(res) == set(A.PROFILE_KINDS)
-    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 13
+    assert all(v == (0.0, 0) for v in res.values()) and len(res) == 14
     assert A.lib().fa_profile_end(None, None) == A.FA_ERR_INVALID_ARG
 
 
@@ -289,7 +290,8 @@ def test_fwd_merge_host_checks():
 
 def test_bwd_stats_and_accumulate_host_checks():
     s = shape()
-    need = A.lib().fa_bwd_workspace_bytes(ctypes.byref(s))
+    with A.bwd_mode("deterministic"):   # the statistics entry points use the separate passes' layout
+        need = A.lib().fa_bwd_workspace_bytes(ctypes.byref(s))
     st = lambda shp, ws=P, nb=need, **kw: A.lib().fa_bwd_stats(  # noqa: E731
         None if shp is None else ctypes.byref(shp), kw.get("o", P), kw.get("do", P), kw.get("lse", P), ws, nb, None)
     assert st(None) == A.FA_ERR_INVALID_ARG
@@ -308,3 +310,34 @@ def test_bwd_stats_and_accumulate_host_checks():
         assert acc(s, **{which: P + 8}) == A.FA_ERR_INVALID_ARG
     assert acc(s, ws=0) == A.FA_ERR_INVALID_ARG
     assert acc(s, nb=need - 1) == A.FA_ERR_INVALID_ARG
+
+
+def test_bwd_mode_setting():
+    """fa_set_bwd_mode validates its argument, fa_get_bwd_mode reads it back, and
+    the workspace size follows the mode (the fused mode adds the fp32 dQ
+    accumulator); no GPU is touched."""
+    L = A.lib()
+    old = L.fa_get_bwd_mode()
+    L.fa_set_bwd_mode(0)
+    try:
+        assert L.fa_set_bwd_mode(3) == A.FA_ERR_INVALID_ARG and L.fa_set_bwd_mode(-1) == A.FA_ERR_INVALID_ARG
+        assert L.fa_get_bwd_mode() == old
+        if os.environ.get("FA_DQ_MODE"):
+            return   # the environment fixes the mode; the sizes below would not follow the setting
+        s = A.make_shape(2, 8, 2, 1000, 128, 0.1, 1)
+        sizes = {}
+        for name, m in A.BWD_MODES.items():
+            assert L.fa_set_bwd_mode(m) == A.FA_OK and L.fa_get_bwd_mode() == m
+            assert A.get_bwd_mode() == name
+            sizes[name] = L.fa_bwd_workspace_bytes(ctypes.byref(s))
+        acc = -(-2 * 8 * 1000 * 128 * 4 // 256) * 256
+        assert sizes["fused"] == sizes["deterministic"] + acc and sizes["auto"] == sizes["fused"]
+        A.set_bwd_mode("auto")
+        with A.bwd_mode("deterministic"):
+            assert A.get_bwd_mode() == "deterministic"
+            s64 = A.make_shape(1, 4, 4, 300, 64, 0.1, 0)
+            small = L.fa_bwd_workspace_bytes(ctypes.byref(s64))
+        assert A.get_bwd_mode() == "auto"
+        assert L.fa_bwd_workspace_bytes(ctypes.byref(s64)) == small   # auto keeps D = 64 on the separate passes
+    finally:
+        L.fa_set_bwd_mode(old)

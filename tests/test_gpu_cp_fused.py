@@ -8,7 +8,9 @@ two key blocks of N keys each (the first "below the diagonal": unmasked, the
 second "on it": causal), exactly the pairs a context-parallel rank computes,
 and the merged / summed results are compared with the oracle's block
 functions joined by its log-sum-exp merge (oracle.attention_forward_block,
-merge_partials, attention_backward_block), at the parity tolerances.
+merge_partials, attention_backward_block), at the parity tolerances.  The
+backward steps run in both backward modes: the fused kernel (default for
+D = 128; dQ reduced straight into the fp32 sum) and the separate passes.
 """
 import math
 
@@ -38,9 +40,15 @@ def _f64(t):
     return t.float().cpu().double().numpy()
 
 
+@pytest.mark.parametrize("mode", ["auto", "deterministic"])
 @pytest.mark.parametrize("B,Hq,Hkv,N,D", [(1, 4, 2, 300, 128), (2, 2, 2, 256, 64), (1, 8, 1, 1000, 128)])
-def test_fused_pair_steps_match_oracle(B, Hq, Hkv, N, D):
+def test_fused_pair_steps_match_oracle(B, Hq, Hkv, N, D, mode):
     dev = _gpu()
+    with A.bwd_mode(mode):
+        _pair_steps(dev, B, Hq, Hkv, N, D)
+
+
+def _pair_steps(dev, B, Hq, Hkv, N, D):
     g = torch.Generator().manual_seed(4000 + N + D)
     q, do = (torch.randn(B, Hq, N, D, generator=g).to(torch.bfloat16) for _ in range(2))
     k0, v0, k1, v1 = (torch.randn(B, Hkv, N, D, generator=g).to(torch.bfloat16) for _ in range(4))

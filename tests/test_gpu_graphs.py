@@ -4,9 +4,11 @@ Launch-bound uses (small problems, one decode step per generated token) want
 the launches captured once and replayed.  Every entry point enqueues only
 kernels on the caller's stream and allocates nothing on the device, so a
 forward + backward step and a decode call can be captured with
-torch.cuda.graph and replayed.  The default path is deterministic, so each
+torch.cuda.graph and replayed.  In the deterministic backward mode each
 replay must equal the eager result bit for bit, also after the inputs are
-overwritten in place between replays.
+overwritten in place between replays; in the fused mode dQ is summed by fp32
+reductions in varying order, so it is held to a tight relative error and
+everything else to bitwise equality.
 """
 import pytest
 import torch
@@ -23,8 +25,26 @@ def _gpu():
     return torch.device("cuda:0")
 
 
-def test_forward_backward_step_replays_bitwise():
+def _rel(a, b):
+    return float((a.float() - b.float()).norm() / b.float().norm().clamp_min(1e-6))
+
+
+def _assert_replay(got_all, ref_all, fused):
+    for i, (got, ref) in enumerate(zip(got_all, ref_all)):
+        if fused and i == 2:   # dq
+            assert _rel(got, ref) <= 2e-3
+        else:
+            assert torch.equal(got, ref)
+
+
+@pytest.mark.parametrize("mode", ["deterministic", "fused"])
+def test_forward_backward_step_replays(mode):
     dev = _gpu()
+    with A.bwd_mode(mode):
+        _step_replays(dev, mode == "fused")
+
+
+def _step_replays(dev, fused):
     wl = Workload("graph", B=1, Hq=4, Hkv=2, N=1000, D=128, causal=True, seed=123)
     q, k, v, do = (x.to(dev) for x in make_inputs(wl))
     o, lse = torch.empty_like(q), torch.empty(1, 4, 1000, device=dev, dtype=torch.float32)
@@ -52,8 +72,7 @@ def test_forward_backward_step_replays_bitwise():
         g.replay()
     torch.cuda.synchronize()
     assert A.device_status(dev) == A.FA_OK
-    for got, ref in zip((o, lse, dq, dk, dv), eager):
-        assert torch.equal(got, ref)
+    _assert_replay((o, lse, dq, dk, dv), eager, fused)
     # new inputs written in place: the replay computes on them
     q.copy_(torch.flip(q, dims=[2]))
     step()
@@ -64,8 +83,7 @@ def test_forward_backward_step_replays_bitwise():
     g.replay()
     torch.cuda.synchronize()
     assert A.device_status(dev) == A.FA_OK
-    for got, ref in zip((o, lse, dq, dk, dv), eager2):
-        assert torch.equal(got, ref)
+    _assert_replay((o, lse, dq, dk, dv), eager2, fused)
     assert not torch.equal(eager2[0], eager[0])
 
 

@@ -89,16 +89,20 @@ def test_small_shapes_full(B, Hq, Hkv, N, D, causal, scale, sqk):
         assert e <= G_TOL, f"{name} rel Frobenius err {e}"
 
 
-@pytest.mark.parametrize("mode", ["atomic", "separate"])
+@pytest.mark.parametrize("mode", ["fused", "separate", "auto"])
 def test_backward_dq_modes(mode):
     """Both dQ strategies (fused kernel with fp32 reductions; separate dQ
-    pass) match the oracle and run the kernels they claim to."""
+    pass), and the default choice between them, match the oracle and run the
+    kernels they claim to."""
     _gpu()
     import os
     import subprocess
     import sys
     here = os.path.dirname(os.path.abspath(__file__))
-    r = subprocess.run([sys.executable, os.path.join(here, "_dq_mode_check.py")], env=dict(os.environ, FA_DQ_MODE=mode),
+    env = {k: v for k, v in os.environ.items() if k != "FA_DQ_MODE"}
+    if mode != "auto":
+        env["FA_DQ_MODE"] = mode
+    r = subprocess.run([sys.executable, os.path.join(here, "_dq_mode_check.py")], env=env,
                        capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout + r.stderr
 
@@ -135,13 +139,33 @@ def test_backward_dkdv_tile_variants(tile):
 
 
 def test_backward_deterministic_separate_mode():
-    """The default backward has no reductions: repeated calls are bitwise equal."""
+    """The deterministic backward has no reductions: repeated calls are bitwise equal."""
     wl = WORKLOADS["tiny"].with_(causal=True, N=700, Hq=4, Hkv=2, D=128)
     q, k, v, do = make_inputs(wl)
-    a = run(q, k, v, do, True, wl.softmax_scale)
-    b = run(q, k, v, do, True, wl.softmax_scale)
+    with A.bwd_mode("deterministic"):
+        a = run(q, k, v, do, True, wl.softmax_scale)
+        b = run(q, k, v, do, True, wl.softmax_scale)
     for t in ("dq", "dk", "dv"):
         assert np.array_equal(a[t], b[t]), t
+
+
+def test_backward_fused_repeats():
+    """The fused backward sums each dQ row over key blocks by fp32 reductions in
+    an order that varies from run to run; dK and dV accumulate inside one CTA
+    and repeat bitwise.  Two runs' dQ agree far inside the parity tolerance,
+    and both modes agree with each other likewise."""
+    wl = WORKLOADS["tiny"].with_(causal=True, N=1000, Hq=8, Hkv=2, D=128)
+    q, k, v, do = make_inputs(wl)
+    with A.bwd_mode("fused"):
+        a = run(q, k, v, do, True, wl.softmax_scale)
+        b = run(q, k, v, do, True, wl.softmax_scale)
+    with A.bwd_mode("deterministic"):
+        c = run(q, k, v, do, True, wl.softmax_scale)
+    for t in ("dk", "dv"):
+        assert np.array_equal(a[t], b[t]), t
+        assert rel_fro(a[t], c[t]) <= 2e-3, t
+    assert rel_fro(a["dq"], b["dq"]) <= 2e-3
+    assert rel_fro(a["dq"], c["dq"]) <= 2e-3
 
 
 def test_repeat_calls_identical_forward():

@@ -7,10 +7,11 @@ region the library reserves statically on each device.  These tests call it
 through the C ABI and check it:
 
   * twice in a row against the regular fa_bwd entry point (which takes a
-    caller workspace).  The default backward has no floating-point reductions
-    in global memory, so the two must agree bit for bit; under the fused mode
-    (FA_DQ_MODE=atomic) dQ is summed in varying order and the parity tolerance
-    applies to it instead;
+    caller workspace) in its deterministic mode.  fa_bwd_noalloc always runs
+    those passes, which have no floating-point reductions in global memory,
+    so the two must agree bit for bit (unless FA_DQ_MODE forces the fused
+    kernel on fa_bwd: then dQ, summed in varying order, is held to the parity
+    tolerance instead);
   * once against the fp64 oracle at the parity tolerances;
   * after a call on a larger shape (ragged N, GQA, more rows of per-row
     statistics and a larger padded length) that leaves its contents in the
@@ -32,7 +33,7 @@ from tiled_attention_16_b200.workloads import Workload, make_inputs
 pytestmark = pytest.mark.gpu
 
 G_TOL = 2e-2
-FUSED = os.environ.get("FA_DQ_MODE") == "atomic"
+FUSED = os.environ.get("FA_DQ_MODE") in ("atomic", "fused")   # the environment fixes fa_bwd's mode
 
 
 def _gpu():
@@ -58,7 +59,8 @@ def assert_same(got, ref, what):
 
 def inputs(dev, B, Hq, Hkv, N, D, causal, seed):
     wl = Workload("noalloc", B=B, Hq=Hq, Hkv=Hkv, N=N, D=D, causal=causal, seed=seed)
-    assert A.workspace_bytes(B, Hq, Hkv, N, D) <= A.NOALLOC_SCRATCH_BYTES
+    with A.bwd_mode("deterministic"):   # the scratch fa_bwd_noalloc needs
+        assert A.workspace_bytes(B, Hq, Hkv, N, D) <= A.NOALLOC_SCRATCH_BYTES
     cpu = make_inputs(wl)
     q, k, v, do = (x.to(dev) for x in cpu)
     o, lse = A.fwd(q, k, v, causal=causal)
@@ -69,7 +71,8 @@ def inputs(dev, B, Hq, Hkv, N, D, causal, seed):
 def test_noalloc_matches_workspace_backward_twice(B, Hq, Hkv, N, D, causal):
     dev = _gpu()
     cpu, (q, k, v, o, do, lse) = inputs(dev, B, Hq, Hkv, N, D, causal, seed=77)
-    ref = A.bwd(q, k, v, o, do, lse, causal=causal)
+    with A.bwd_mode("deterministic"):
+        ref = A.bwd(q, k, v, o, do, lse, causal=causal)
     for call in range(2):
         got = A.bwd_noalloc(q, k, v, o, do, lse, causal=causal)
         assert A.device_status(dev) == A.FA_OK, f"call {call}: sites {A.timeout_sites():#x}"
@@ -91,8 +94,9 @@ def test_noalloc_after_larger_shape():
     small = (1, 3, 1, 257, 128, True)     # MQA, Npad 384, ragged last tile
     _, tb = inputs(dev, *big, seed=91)
     _, ts = inputs(dev, *small, seed=92)
-    ref_small = A.bwd(*ts, causal=True)
-    ref_big = A.bwd(*tb, causal=True)
+    with A.bwd_mode("deterministic"):
+        ref_small = A.bwd(*ts, causal=True)
+        ref_big = A.bwd(*tb, causal=True)
     for rnd in range(2):
         got_big = A.bwd_noalloc(*tb, causal=True)
         got_small = A.bwd_noalloc(*ts, causal=True)
@@ -104,7 +108,8 @@ def test_noalloc_after_larger_shape():
 def test_noalloc_rejects_oversized_problem():
     dev = _gpu()
     B, H, N, D = 1, 64, 81920, 64  # row statistics alone: 2 x 64 x 81920 x 4 B = 40 MiB
-    assert A.workspace_bytes(B, H, H, N, D) > A.NOALLOC_SCRATCH_BYTES
+    with A.bwd_mode("deterministic"):
+        assert A.workspace_bytes(B, H, H, N, D) > A.NOALLOC_SCRATCH_BYTES
     x = torch.zeros(B, H, N, D, device=dev, dtype=torch.bfloat16)
     lse = torch.zeros(B, H, N, device=dev, dtype=torch.float32)
     with pytest.raises(A.FAError) as ei:

@@ -8,6 +8,7 @@ device is not a B200 the calls raise.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import math
 import os
@@ -91,6 +92,10 @@ def lib() -> ctypes.CDLL:
         L.fa_profile_begin.restype = ctypes.c_int
         L.fa_profile_end.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(ctypes.c_int)]
         L.fa_profile_end.restype = ctypes.c_int
+        L.fa_set_bwd_mode.argtypes = [ctypes.c_int]
+        L.fa_set_bwd_mode.restype = ctypes.c_int
+        L.fa_get_bwd_mode.argtypes = []
+        L.fa_get_bwd_mode.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -241,6 +246,35 @@ def decode(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = Tru
     if st != FA_OK:
         raise FAError(st, "fa_decode")
     return out, lse
+
+
+BWD_MODES = {"auto": 0, "deterministic": 1, "fused": 2}   # FA_BWD_AUTO, _DETERMINISTIC, _FUSED
+
+
+def set_bwd_mode(mode: str) -> None:
+    """Process-wide dQ strategy of bwd(): "fused" (one kernel, dQ summed by fp32
+    reductions in varying order), "deterministic" (separate dQ pass; repeated
+    calls bitwise equal) or "auto" (the measured choice: fused for D = 128).
+    The environment variable FA_DQ_MODE, if set, overrides it."""
+    st = lib().fa_set_bwd_mode(BWD_MODES[mode])
+    if st != FA_OK:
+        raise FAError(st, "fa_set_bwd_mode")
+
+
+def get_bwd_mode() -> str:
+    m = lib().fa_get_bwd_mode()
+    return next(k for k, v in BWD_MODES.items() if v == m)
+
+
+@contextlib.contextmanager
+def bwd_mode(mode: str):
+    """Run the enclosed calls under backward mode `mode`, then restore the previous one."""
+    old = get_bwd_mode()
+    set_bwd_mode(mode)
+    try:
+        yield
+    finally:
+        set_bwd_mode(old)
 
 
 def workspace_bytes(B, Hq, Hkv, N, D, causal=False, scale=None) -> int:
@@ -452,7 +486,7 @@ def timeout_sites() -> int:
 PROFILE_KINDS = ("fa_fwd_kernel", "fa_bwd_preprocess", "fa_bwd_kernel", "fa_bwd_dq_convert",
                  "fa_bwd_dkdv_kernel", "fa_bwd_dq_kernel", "fa_fwd_fp8_kernel", "fa_decode",
                  "fa_lse_merge_kernel", "fa_accumulate_kernel", "fa_fwd_pair_kernel",
-                 "fa_bwd_dkdv_pair_kernel", "fa_bwd_dq_pair_kernel")
+                 "fa_bwd_dkdv_pair_kernel", "fa_bwd_dq_pair_kernel", "fa_bwd_fused_kernel")
 
 
 def profile_begin() -> None:

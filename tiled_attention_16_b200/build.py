@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa_sm100.so")
-SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_fwd_pair.cu", "fa_fwd_fp8.cu", "fa_bwd.cu", "fa_bwd_split.cu", "fa_bwd_pair.cu", "fa_decode.cu", "fa_cp.cu", "fa_selftest.cu"]
+SOURCES = ["fa_api.cu", "fa_fwd.cu", "fa_fwd_pair.cu", "fa_fwd_fp8.cu", "fa_bwd.cu", "fa_bwd_split.cu", "fa_bwd_fused.cu", "fa_bwd_pair.cu", "fa_decode.cu", "fa_cp.cu", "fa_selftest.cu"]
 HEADERS = ["sm100.cuh", "fa_internal.h"]
 
 NVCC_FLAGS = [

@@ -8,6 +8,7 @@
 #include <cstdlib>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <utility>
 #include <vector>
@@ -198,17 +199,27 @@ bool fwd_use_pair(const fa_shape& s) {
     return s.N >= kPairMinN;
 }
 
-// dQ strategy of the backward: a separate dQ pass (default; deterministic, no
-// reductions) or the fused kernel with fp32 reductions ("atomic").  Chosen by
-// measurement; FA_DQ_MODE=atomic|separate overrides it (read once).
-bool dq_separate_mode() {
-    static int mode = -1;
+// dQ strategy of the backward (FA_BWD_AUTO / _DETERMINISTIC / _FUSED): the
+// process-wide choice of fa_set_bwd_mode, unless the environment variable
+// FA_DQ_MODE=separate|fused (or its older name atomic; read once) fixes it.
+// AUTO is the measured choice: the fused kernel for D = 128, the separate
+// passes for D = 64.
+std::atomic<int> g_bwd_mode{FA_BWD_AUTO};
+int env_bwd_mode() {
+    static int mode = FA_BWD_AUTO;
     static std::once_flag once;
     std::call_once(once, [] {
         const char* e = std::getenv("FA_DQ_MODE");
-        mode = (e && std::strcmp(e, "atomic") == 0) ? 0 : 1;
+        if (e && (std::strcmp(e, "atomic") == 0 || std::strcmp(e, "fused") == 0)) mode = FA_BWD_FUSED;
+        else if (e && std::strcmp(e, "separate") == 0) mode = FA_BWD_DETERMINISTIC;
     });
-    return mode == 1;
+    return mode;
+}
+bool bwd_fused(const fa_shape& s) {
+    int m = env_bwd_mode();
+    if (m == FA_BWD_AUTO) m = g_bwd_mode.load(std::memory_order_relaxed);
+    if (m == FA_BWD_AUTO) return s.D == 128;
+    return m == FA_BWD_FUSED;
 }
 
 // Scratch of fa_bwd_noalloc: reserved statically in device memory on every
@@ -489,7 +500,7 @@ fa_status fa_decode(const fa_kv_shape* shape, const void* q, const void* k, cons
 
 size_t fa_bwd_workspace_bytes(const fa_shape* shape) {
     if (check_shape(shape) != FA_OK) return 0;
-    return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total;
+    return bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, bwd_fused(*shape)).total;
 }
 
 }  // extern "C"
@@ -499,7 +510,7 @@ namespace {
 // What bwd_impl runs: the whole backward (fa_bwd), only the row statistics
 // into the workspace (fa_bwd_stats), or the two passes on statistics already
 // in the workspace, adding into fp32 sums (fa_bwd_accumulate).
-enum BwdMode { kBwdFull, kBwdStats, kBwdAccumulate };
+enum BwdMode { kBwdFull, kBwdFullDeterministic, kBwdStats, kBwdAccumulate };
 struct AccArgs {
     float* dq;
     float* dk;
@@ -514,15 +525,20 @@ fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const voi
     if (st != FA_OK) return st;
     const bool need_stats_in = mode != kBwdAccumulate;
     const bool need_passes = mode != kBwdStats;
+    const bool full = mode == kBwdFull || mode == kBwdFullDeterministic;
     if (need_stats_in && (!aligned16(o) || !aligned16(dout) || !aligned4(lse))) return FA_ERR_INVALID_ARG;
     if (need_passes && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dout))) return FA_ERR_INVALID_ARG;
-    if (mode == kBwdFull && (!aligned16(dq) || !aligned16(dk) || !aligned16(dv))) return FA_ERR_INVALID_ARG;
+    if (full && (!aligned16(dq) || !aligned16(dk) || !aligned16(dv))) return FA_ERR_INVALID_ARG;
     if (mode == kBwdAccumulate && (!acc || !aligned16(acc->dq) || !aligned16(acc->dk) || !aligned16(acc->dv)))
         return FA_ERR_INVALID_ARG;
     const fa_shape& s = *shape;
-    // the statistics entry points always use the separate passes' layout
-    const bool separate = mode != kBwdFull || dq_separate_mode();
-    const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D, !separate);
+    // The fused kernel runs for fa_bwd when the backward mode selects it, and
+    // for fa_bwd_accumulate too when D = 128 (dQ then goes straight into the
+    // caller's fp32 sum); the workspace holds the fp32 dQ accumulator only for
+    // fa_bwd, so the statistics entry points share the separate passes' layout.
+    const bool fused = (mode == kBwdFull && bwd_fused(s)) || (mode == kBwdAccumulate && s.D == 128 && bwd_fused(s));
+    const bool separate = !fused;
+    const BwdWorkspace ws = bwd_workspace_layout(s.B, s.Hq, s.N, s.D, fused && mode == kBwdFull);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < ws.total)
         return FA_ERR_INVALID_ARG;
     if ((st = check_device()) != FA_OK) return st;
@@ -531,8 +547,8 @@ fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const voi
                         !make_map(&tv, v, s.B * s.Hkv, s.N, s.D) || !make_map(&tdo, dout, s.B * s.Hq, s.N, s.D)))
         return FA_ERR_CUDA;
     // the accumulate epilogues live in the one-CTA passes
-    const bool pair_dkdv = mode == kBwdFull && separate && bwd_dkdv_use_pair(s);
-    const bool pair_dq = mode == kBwdFull && separate && bwd_dq_use_pair(s);
+    const bool pair_dkdv = full && separate && bwd_dkdv_use_pair(s);
+    const bool pair_dq = full && separate && bwd_dq_use_pair(s);
     CUtensorMap tq_half, tdo_half, tk_half, tv_half;
     if (pair_dkdv && (!make_map(&tq_half, q, s.B * s.Hq, s.N, s.D, 2, kTileM / 2) ||
                       !make_map(&tdo_half, dout, s.B * s.Hq, s.N, s.D, 2, kTileM / 2)))
@@ -570,7 +586,7 @@ fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const voi
     p.scale_log2 = static_cast<float>(static_cast<double>(s.scale) * 1.4426950408889634);
     p.lse2 = reinterpret_cast<const float*>(wsb + ws.lse2_off);
     p.dvec = reinterpret_cast<const float*>(wsb + ws.dvec_off);
-    p.dq_acc = separate ? nullptr : reinterpret_cast<float*>(wsb + ws.dq_off);
+    p.dq_acc = (fused && mode == kBwdFull) ? reinterpret_cast<float*>(wsb + ws.dq_off) : nullptr;
     p.dq = dq;
     p.dk = dk;
     p.dv = dv;
@@ -587,7 +603,7 @@ fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const voi
     if (need_stats_in) {
         e = timed(1, strm, [&] {
             return launch_bwd_preprocess(s.D, o, dout, lse, reinterpret_cast<float*>(wsb + ws.lse2_off),
-                                         reinterpret_cast<float*>(wsb + ws.dvec_off), separate ? nullptr : p.dq_acc,
+                                         reinterpret_cast<float*>(wsb + ws.dvec_off), p.dq_acc,
                                          s.B * s.Hq, s.N, Npad, s.scale,
                                          reinterpret_cast<unsigned int*>(wsb + ws.sched_off), strm);
         });
@@ -604,8 +620,14 @@ fa_status bwd_impl(BwdMode mode, const fa_shape* shape, const void* q, const voi
             e = pair_dq ? timed(12, strm, [&] { return launch_bwd_dq_pair(tq, tk, tk_half, tv_half, tdo, p, strm); })
                      : timed(5, strm, [&] { return launch_bwd_dq(s.D, tq, tk, tv, tdo, p, strm); });
     } else {
-        if (e == cudaSuccess) e = timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
+        // accumulate mode: the kernel's reductions add into the caller's dQ sum,
+        // which a first call clears
+        if (e == cudaSuccess && mode == kBwdAccumulate && acc->first_dq)
+            e = cudaMemsetAsync(acc->dq, 0, static_cast<size_t>(s.B) * s.Hq * s.N * s.D * sizeof(float), strm);
         if (e == cudaSuccess)
+            e = s.D == 128 ? timed(13, strm, [&] { return launch_bwd_fused(tq, tk, tv, tdo, p, strm); })
+                           : timed(2, strm, [&] { return launch_bwd_main(s.D, tq, tk, tv, tdo, p, strm); });
+        if (e == cudaSuccess && mode == kBwdFull)
             e = timed(3, strm, [&] {
                 return launch_bwd_dq_convert(p.dq_acc, dq, static_cast<size_t>(s.B) * s.Hq * s.N * s.D, strm);
             });
@@ -647,14 +669,22 @@ fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k, co
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) || !aligned4(lse) ||
         !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
         return FA_ERR_INVALID_ARG;
-    if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, !dq_separate_mode()).total >
-        FA_NOALLOC_SCRATCH_BYTES)
+    if (bwd_workspace_layout(shape->B, shape->Hq, shape->N, shape->D, false).total > FA_NOALLOC_SCRATCH_BYTES)
         return FA_ERR_TOO_LARGE;
     if ((st = check_device()) != FA_OK) return st;
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != FA_OK) return st;
-    return fa_bwd(shape, q, k, v, o, dout, lse, dq, dk, dv, scratch, FA_NOALLOC_SCRATCH_BYTES, stream);
+    return bwd_impl(kBwdFullDeterministic, shape, q, k, v, o, dout, lse, dq, dk, dv, nullptr, scratch,
+                    FA_NOALLOC_SCRATCH_BYTES, stream);
 }
+
+fa_status fa_set_bwd_mode(int mode) {
+    if (mode != FA_BWD_AUTO && mode != FA_BWD_DETERMINISTIC && mode != FA_BWD_FUSED) return FA_ERR_INVALID_ARG;
+    g_bwd_mode.store(mode, std::memory_order_relaxed);
+    return FA_OK;
+}
+
+int fa_get_bwd_mode(void) { return g_bwd_mode.load(std::memory_order_relaxed); }
 
 fa_status fa_lse_merge(long long rows, int D, const void* o_part, const float* lse_part, float* o_acc,
                        float* lse_acc, void* o_out, int first, void* stream) {

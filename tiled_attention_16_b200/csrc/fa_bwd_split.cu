@@ -62,21 +62,6 @@ __host__ __device__ constexpr uint32_t packed_col(int kk) {
     return static_cast<uint32_t>((kk / (kCols / 16)) * kCols + (kk % (kCols / 16)) * 8);
 }
 
-// acc[0..15] = (first ? 0 : acc[0..15]) + the 16 fp32 values in v (one
-// thread's row segment; 16-byte accesses).
-__device__ __forceinline__ void accumulate16(float* acc, const uint32_t (&v)[16], int first) {
-    float4* a4 = reinterpret_cast<float4*>(acc);
-#pragma unroll
-    for (int t = 0; t < 4; ++t) {
-        float4 a = first ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[t];
-        a.x += __uint_as_float(v[4 * t]);
-        a.y += __uint_as_float(v[4 * t + 1]);
-        a.z += __uint_as_float(v[4 * t + 2]);
-        a.w += __uint_as_float(v[4 * t + 3]);
-        a4[t] = a;
-    }
-}
-
 __device__ __forceinline__ void wait_drain(uint64_t* bar, uint32_t parity, int site) {
     if (mbar_try_wait(bar, parity)) return;
     unsigned long long t0 = globaltimer_ns();

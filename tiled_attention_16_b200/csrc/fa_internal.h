@@ -114,6 +114,9 @@ cudaError_t launch_bwd_preprocess(int D, const void* o, const void* dout, const 
                                   cudaStream_t stream);
 
 // Fused backward: dK, dV and dQ (fp32 reductions into p.dq_acc).
+// the persistent fused backward (D = 128): dK, dV and dQ partials in one pass
+cudaError_t launch_bwd_fused(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
 cudaError_t launch_bwd_main(int D, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const BwdParams& p, cudaStream_t stream);
 

@@ -111,6 +111,20 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
         : "memory");
 }
 
+// dst (global) += src (shared), element-wise in fp32, applied in L2 by the
+// bulk copy engine (cp.reduce.async.bulk .add.f32).  Both addresses 16-byte
+// aligned, bytes a multiple of 16.  Completion is tracked per issuing thread
+// in bulk async-groups: bulk_commit_group closes a group, bulk_wait_read_all
+// returns once the shared-memory sources of all this thread's groups have
+// been read, bulk_wait_all once the groups have completed.
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+                 ::"l"(dst), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // tcgen05: tensor memory
 // ----------------------------------------------------------------------------
@@ -444,6 +458,21 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // Byte offset of element (row, col) inside a 128-byte-swizzled K-major tile
 // made of 64-column atoms of `rows` rows each (atom a holds columns
 // [64a, 64a+64)); the 16-byte chunk index is XORed with row % 8.
+// acc[0..15] = (first ? 0 : acc[0..15]) + the 16 fp32 values in v (one
+// thread's row segment of a TMEM load; 16-byte accesses).
+__device__ __forceinline__ void accumulate16(float* acc, const uint32_t (&v)[16], int first) {
+    float4* a4 = reinterpret_cast<float4*>(acc);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        float4 a = first ? make_float4(0.f, 0.f, 0.f, 0.f) : a4[t];
+        a.x += __uint_as_float(v[4 * t]);
+        a.y += __uint_as_float(v[4 * t + 1]);
+        a.z += __uint_as_float(v[4 * t + 2]);
+        a.w += __uint_as_float(v[4 * t + 3]);
+        a4[t] = a;
+    }
+}
+
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col, uint32_t rows) {
     uint32_t atom = col >> 6;
     uint32_t c = col & 63u;
