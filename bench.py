@@ -24,6 +24,7 @@ import os
 import statistics
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -105,6 +106,74 @@ class ClockSampler:
         if not sm:
             return None
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class NvmlClockSampler:
+    """SM clock and clock-event reasons read through NVML every `period_s` from a
+    background thread (read-only queries; nothing on the GPU is changed).  A
+    20-step timed region lasts about 0.1 s, too short for nvidia-smi's
+    100 ms loop, so this is the sampler the bench uses where NVML loads;
+    ClockSampler (nvidia-smi) is the fallback.  `nvml` may be a stand-in
+    module (tests)."""
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
+
+    def __init__(self, pci_bus_id: str | None = None, index: int = 0, period_s: float = 0.005, nvml=None):
+        self.bus, self.index, self.period = pci_bus_id, index, period_s
+        self.nv = nvml
+        self.samples = []    # (host time, SM MHz, reason bits)
+        self.window = None
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    def start(self) -> bool:
+        try:
+            if self.nv is None:
+                import pynvml
+                self.nv = pynvml
+            nv = self.nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByPciBusId(self.bus) if self.bus else nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:   # no NVML, no device: the caller falls back to nvidia-smi
+            return False
+
+        def run():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                         int(reasons(h))))
+                except Exception:
+                    return
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
+        return True
+
+    def stop(self):
+        if self._thread is None:
+            return None
+        self._stop.set()
+        self._thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        got = [s for s in self.samples if self.window is None or self.window[0] <= s[0] <= self.window[1]]
+        if not got:
+            return None
+        bits = 0
+        for s in got:
+            bits |= s[2]
+        return {"sm_mhz": statistics.median(s[1] for s in got), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(n for n, b in self.REASON_BITS.items() if bits & b), "samples": len(got),
+                "source": f"nvml every {self.period * 1e3:.0f} ms"}
 
 
 # ----------------------------------------------------------------------------- traffic record
@@ -287,9 +356,12 @@ def run_gpu(args, wl):
     if A.device_status(dev) != A.FA_OK:
         raise RuntimeError(f"device status not OK after warm-up (sites {A.timeout_sites():#x})")
 
-    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
-    sampler.start()
-    time.sleep(0.3)
+    props = torch.cuda.get_device_properties(dev)
+    sampler = NvmlClockSampler(f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0")
+    if not sampler.start():
+        sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+        sampler.start()
+        time.sleep(0.3)
     stream = torch.cuda.current_stream(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:

@@ -64,6 +64,62 @@ def test_clock_sampler_with_no_process():
     assert bench.ClockSampler(0).stop() is None
 
 
+class _FakeNvml:
+    """Read-only NVML stand-in: a clock that steps through `mhz` and the
+    sw_power_cap reason bit from the third sample on."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, mhz, fail_init=False):
+        self.mhz, self.n, self.fail, self.calls = list(mhz), 0, fail_init, []
+
+    def nvmlInit(self):
+        if self.fail:
+            raise RuntimeError("no NVML")
+
+    def nvmlShutdown(self):
+        self.calls.append("shutdown")
+
+    def nvmlDeviceGetHandleByPciBusId(self, bus):
+        self.calls.append(bus)
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        v = self.mhz[min(self.n, len(self.mhz) - 1)]
+        self.n += 1
+        return v
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return 0x4 if self.n >= 3 else 0
+
+
+def test_nvml_clock_sampler_keeps_window_samples_and_reasons():
+    nv = _FakeNvml([1965, 1965, 1800, 1700, 1700])
+    cs = bench.NvmlClockSampler("00000000:1b:00.0", period_s=0.001, nvml=nv)
+    t0 = time.time()
+    assert cs.start()
+    time.sleep(0.05)
+    cs.mark(t0 - 1.0, time.time() + 1.0)
+    got = cs.stop()
+    assert nv.calls[0] == "00000000:1b:00.0" and nv.calls[-1] == "shutdown"
+    assert got["samples"] >= 5 and got["sm_max_mhz"] == 1965.0 and got["sm_mhz"] == 1700.0
+    assert got["reasons"] == ["sw_power_cap"] and got["source"].startswith("nvml")
+    # a window that holds no sample gives no record
+    cs2 = bench.NvmlClockSampler(None, period_s=0.001, nvml=_FakeNvml([1965]))
+    cs2.nv.nvmlDeviceGetHandleByIndex = lambda i: "h"
+    assert cs2.start()
+    time.sleep(0.01)
+    cs2.mark(0.0, 1.0)
+    assert cs2.stop() is None
+
+
+def test_nvml_clock_sampler_reports_failure_to_start():
+    cs = bench.NvmlClockSampler("x", nvml=_FakeNvml([1], fail_init=True))
+    assert cs.start() is False and cs.stop() is None
+
+
 def test_traffic_record_follows_the_source_hash(tmp_path, monkeypatch):
     k = "fa_fwd_kernel"
     h = bench.kernel_source_hash(k)
