@@ -507,35 +507,47 @@ def run_gpu(args, wl):
             co, clse = A.fwd(cq, ck, cv, causal=cwl.causal)
             A.bwd(cq, ck, cv, co, cdo, clse, causal=cwl.causal, workspace=cws)
 
-        def timed_ms(fn, n):
-            for _ in range(3):
-                fn()
-            torch.cuda.synchronize()
+        def timed_once(fn):
             t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             t0.record()
-            for _ in range(n):
-                fn()
+            fn()
             t1.record()
             torch.cuda.synchronize()
-            return t0.elapsed_time(t1) / n
+            return t0.elapsed_time(t1)
 
+        # Each leg runs ~70 ms, long enough for the power cap to move the SM
+        # clock between runs, so the two legs are timed interleaved, in
+        # alternating order, and compared by their medians: both see the same
+        # power state.
         n_cp = 5
-        mono_ms = timed_ms(mono_step, n_cp)
+        for _ in range(2):
+            mono_step()
+            ring_step()
+        torch.cuda.synchronize()
+        mono_runs, cp_runs = [], []
+        for i in range(n_cp):
+            legs = [(mono_runs, mono_step), (cp_runs, ring_step)]
+            for runs, fn in (legs if i % 2 == 0 else legs[::-1]):
+                runs.append(timed_once(fn))
+        mono_ms, cp_ms = statistics.median(mono_runs), statistics.median(cp_runs)
+        # one more ring step under the per-kernel profiler (launch count, merge
+        # and accumulate time), outside the timed runs
         A.profile_begin()
-        cp_ms = timed_ms(ring_step, n_cp)
+        ring_step()
         cp_kernels = A.profile_end()
         if A.device_status(dev) != A.FA_OK:
             raise RuntimeError("device status not OK after the context-parallel ring")
         cflops = cwl.flops_fwd() + cwl.flops_bwd()
         cp_tf = cflops / (cp_ms * 1e-3) / 1e12
         mono_tf = cflops / (mono_ms * 1e-3) / 1e12
-        n_all = n_cp + 3
+        n_all = 1
         breakdown["context_parallel"] = {
             "workload": f"{cwl.name}: B={cwl.B} Hq={cwl.Hq} Hkv={cwl.Hkv} N={cwl.N} D={cwl.D}"
                         f"{' causal' if cwl.causal else ''}",
             "ranks": R, "chunk_rows": cwl.N // (2 * R), "layout": "zigzag",
             "ms_per_step": cp_ms, "tflops": cp_tf, "single_kernel_ms": mono_ms, "single_kernel_tflops": mono_tf,
-            "vs_single_kernel": cp_tf / mono_tf,
+            "vs_single_kernel": cp_tf / mono_tf, "timing": f"{n_cp} runs of each leg interleaved in alternating order; medians",
+            "runs_ms": {"ring": cp_runs, "single_kernel": mono_runs},
             "merge_ms": cp_kernels["fa_lse_merge_kernel"][0] / n_all,
             "accumulate_ms": cp_kernels["fa_accumulate_kernel"][0] / n_all,
             "launches_per_step": sum(nn for _, nn in cp_kernels.values()) / n_all,

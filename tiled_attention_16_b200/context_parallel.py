@@ -37,6 +37,7 @@ float64 reference arithmetic on CPU); there is no fallback when it is not.
 """
 from __future__ import annotations
 
+import functools
 import math
 from typing import Sequence
 
@@ -160,6 +161,39 @@ def _check_shards(q, k, v):
         raise ValueError("q [2,B,Hq,C,D] and k, v [2,B,Hkv,C,D] must agree")
 
 
+class _Lanes:
+    """Two CUDA streams on which the pairs of one ring step that write disjoint
+    sums run side by side, so the last, partly filled wave of one pair's
+    persistent launch overlaps the start of the other lane's launch.  A step
+    runs in rounds; each round forks both lanes from the current stream and
+    joins them back into it.  With CPU tensors (the float64 reference ops of
+    the tests) the calls simply run in order."""
+
+    def __init__(self, like: torch.Tensor):
+        self.streams = [torch.cuda.Stream(like.device), torch.cuda.Stream(like.device)] if like.is_cuda else None
+
+    def run(self, rounds):
+        """rounds: [[calls of lane 0, calls of lane 1], ...]"""
+        if self.streams is None:
+            for rnd in rounds:
+                for lane in rnd:
+                    for f in lane:
+                        f()
+            return
+        cur = torch.cuda.current_stream(self.streams[0].device)
+        for rnd in rounds:
+            for st, lane in zip(self.streams, rnd):
+                if not lane:
+                    continue
+                st.wait_stream(cur)
+                with torch.cuda.stream(st):
+                    for f in lane:
+                        f()
+            for st, lane in zip(self.streams, rnd):
+                if lane:
+                    cur.wait_stream(st)
+
+
 def _last_use(plans) -> dict[int, tuple[int, int]]:
     last = {}
     for s, (_, pairs) in enumerate(plans):
@@ -181,12 +215,17 @@ class _FwdRank:
         self.lse = ops.empty_acc(q.shape[:-1], q)
         self.out = torch.empty_like(q)
         self.started = [False, False]
+        self.lanes = _Lanes(q)
 
     def step(self, s, k_cur, v_cur):
+        # the pairs of query chunk qs fold into its own running result: lane qs
+        lanes = [[], []]
         for i, (qs, ks, cflag) in enumerate(self.plans[s][1]):
-            self.ops.fwd_merge(self.q[qs], k_cur[ks], v_cur[ks], cflag, self.scale, self.o_acc[qs], self.lse[qs],
-                               first=not self.started[qs], out=self.out[qs] if self.last[qs] == (s, i) else None)
+            lanes[qs].append(functools.partial(
+                self.ops.fwd_merge, self.q[qs], k_cur[ks], v_cur[ks], cflag, self.scale, self.o_acc[qs],
+                self.lse[qs], first=not self.started[qs], out=self.out[qs] if self.last[qs] == (s, i) else None))
             self.started[qs] = True
+        self.lanes.run([lanes])
 
 
 class _BwdRank:
@@ -202,20 +241,33 @@ class _BwdRank:
         self.dq_acc = ops.empty_acc(q.shape, q)
         self.dq = torch.empty_like(q)
         self.started = [False, False]
+        self.lanes = _Lanes(q)
 
     def step(self, s, k_cur, v_cur, dk_acc, dv_acc):
         """Step s's pairs: dQ into the local sums, dK/dV into the sums of the
-        shard this rank holds (fresh at step 0, when the shard is its own)."""
+        shard this rank holds (fresh at step 0, when the shard is its own).
+        Pair (qs, ks) writes the sums of query chunk qs and key chunk ks, so
+        the pairs run in two rounds, (0,0) beside (1,1), then (0,1) beside
+        (1,0): lane qs, and no two pairs of a round share a sum.  The first /
+        last flags follow that execution order."""
+        pairs = self.plans[s][1]
+        order = [e for r in (0, 1) for e in enumerate(pairs) if (e[1][0] + e[1][1]) % 2 == r]
+        final = {qs: max(pos for pos, (_, (q2, _, _)) in enumerate(order) if q2 == qs)
+                 for qs in (0, 1) if self.last[qs][0] == s}
+        rounds = [[[], []], [[], []]]
         touched = [False, False]
-        for i, (qs, ks, cflag) in enumerate(self.plans[s][1]):
-            fresh = s == 0 and not touched[ks]
-            self.ops.bwd_accumulate(self.q[qs], k_cur[ks], v_cur[ks], self.do[qs], self.prep[qs], cflag, self.scale,
-                                    self.dq_acc[qs], dk_acc[ks], dv_acc[ks], first_dq=not self.started[qs],
-                                    first_dkv=fresh)
+        for pos, (i, (qs, ks, cflag)) in enumerate(order):
+            lane = rounds[(qs + ks) % 2][qs]
+            lane.append(functools.partial(
+                self.ops.bwd_accumulate, self.q[qs], k_cur[ks], v_cur[ks], self.do[qs], self.prep[qs], cflag,
+                self.scale, self.dq_acc[qs], dk_acc[ks], dv_acc[ks], first_dq=not self.started[qs],
+                first_dkv=s == 0 and not touched[ks]))
             self.started[qs] = True
             touched[ks] = True
-            if self.last[qs] == (s, i):
-                self.ops.accumulate(self.dq_acc[qs], None, first=False, out=self.dq[qs])
+            if final.get(qs) == pos:
+                lane.append(functools.partial(self.ops.accumulate, self.dq_acc[qs], None, first=False,
+                                              out=self.dq[qs]))
+        self.lanes.run(rounds)
         if s == 0:
             for ks in (0, 1):
                 if not touched[ks]:
