@@ -34,7 +34,7 @@ constexpr int kFwdThreads = 320;
 constexpr int kStages = 2;
 constexpr float kRescaleThreshold = 8.0f;
 
-enum FwdSite { kSiteQ = 0, kSiteK = 1, kSiteV = 2, kSiteKVEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteDrain = 7 };
+enum FwdSite { kSiteQ = 0, kSiteK = 1, kSiteKVEmpty = 3, kSiteS = 4, kSiteP = 5, kSiteO = 6, kSiteDrain = 7 };
 
 template <int D>
 struct FwdLayout {
@@ -44,7 +44,7 @@ struct FwdLayout {
     static constexpr int kK = kQ + 2 * kTileBytes;      // kStages tiles
     static constexpr int kV = kK + kStages * kTileBytes;
     static constexpr int kBar = kV + kStages * kTileBytes;
-    static constexpr int kNumBars = 1 + 3 * kStages + 3 * 2 + 1 + 1 + 2 * 2;  // ... drain, q_empty, unit ring
+    static constexpr int kNumBars = 1 + 2 * kStages + 3 * 2 + 1 + 1 + 2 * 2;  // q, K/V full + empty, S/P/O, drain, q_empty, unit ring
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024 B
@@ -188,10 +188,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;                 // [kStages]
-    uint64_t* v_full = bars + 1 + kStages;       // [kStages]
-    uint64_t* kv_empty = bars + 1 + 2 * kStages; // [kStages]
-    uint64_t* s_full = bars + 1 + 3 * kStages;   // [2]
+    // [kStages] K and V of a stage land on one barrier: the MMA thread waits
+    // once per key tile (a completed wait still idles the tensor core for
+    // about 150 cycles, the tcgen05 issue queue being shallow)
+    uint64_t* k_full = bars + 1;
+    uint64_t* kv_empty = bars + 1 + kStages;     // [kStages]
+    uint64_t* s_full = bars + 1 + 2 * kStages;   // [2]
     uint64_t* p_full = s_full + 2;               // [2]
     uint64_t* o_full = p_full + 2;               // [2]
     uint64_t* drain = o_full + 2;
@@ -211,7 +213,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
         mbar_init(q_empty, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&k_full[s], 1);
-            mbar_init(&v_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -273,13 +274,12 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     if (gk >= kStages &&
                         !(ok = mbar_wait(&kv_empty[st], ((gk >> 1) - 1) & 1, abort_flag, kSiteKVEmpty)))
                         break;
-                    mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                    mbar_arrive_expect_tx(&k_full[st], 2 * L::kTileBytes);
                     for (int a = 0; a < D / 64; ++a)
                         tma_load_3d(smem + L::kK + st * L::kTileBytes + a * L::kAtomBytes, &tmK, &k_full[st], a * 64,
                                     j * kTileN, w.kvh);
-                    mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
                     for (int a = 0; a < D / 64; ++a)
-                        tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &v_full[st], a * 64,
+                        tma_load_3d(smem + L::kV + st * L::kTileBytes + a * L::kAtomBytes, &tmV, &k_full[st], a * 64,
                                     j * kTileN, w.kvh);
                     n_kv = gk + 1;
                 }
@@ -292,7 +292,6 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
             if (n_q > 0) mbar_wait_drain(q_full, (n_q - 1) & 1, kSiteDrain);
             for (int k = (n_kv > kStages ? n_kv - kStages : 0); k < n_kv; ++k) {
                 mbar_wait_drain(&k_full[k & 1], (k >> 1) & 1, kSiteDrain);
-                mbar_wait_drain(&v_full[k & 1], (k >> 1) & 1, kSiteDrain);
             }
         }
     } else if (warp == 8) {
@@ -343,8 +342,11 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                 for (int j = 0; j < n_iter; ++j) {
                     const int G = gk + j;
                     const int st = G & 1;
-                    const uint32_t ph = (G >> 1) & 1;
-                    if (!(ok = mbar_wait(&v_full[st], ph, abort_flag, kSiteV))) break;
+                    // V(G) arrived with K(G), whose barrier was waited for before
+                    // S(j) (at the unit start or in the previous iteration); the
+                    // next tile's barrier is waited for once, before the first
+                    // S(j+1)
+                    bool next_kv = false;
                     if (j < nkv[0]) {
                         if (!(ok = mbar_wait(&p_full[0], (c0 + j) & 1, abort_flag, kSiteP))) break;
                         tc_fence_after();
@@ -352,6 +354,7 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                         if (j == nkv[0] - 1) tc_commit(&o_full[0]);
                         if (j + 1 < nkv[0]) {
                             if (!(ok = mbar_wait(&k_full[st ^ 1], ((G + 1) >> 1) & 1, abort_flag, kSiteK))) break;
+                            next_kv = true;
                             tc_fence_after();
                             issue_s(0, st ^ 1);
                             tc_commit(&s_full[0]);
@@ -365,7 +368,8 @@ fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ C
                     }
                     tc_commit(&kv_empty[st]);
                     if (j + 1 < nkv[1]) {
-                        if (!(ok = mbar_wait(&k_full[st ^ 1], ((G + 1) >> 1) & 1, abort_flag, kSiteK))) break;
+                        if (!next_kv && !(ok = mbar_wait(&k_full[st ^ 1], ((G + 1) >> 1) & 1, abort_flag, kSiteK)))
+                            break;
                         tc_fence_after();
                         issue_s(1, st ^ 1);
                         tc_commit(&s_full[1]);
