@@ -38,7 +38,7 @@ constexpr int kF8D = 128;
 constexpr float kF8RescaleThreshold = 8.0f;
 
 // wait sites: the bits of the bf16 forward (a timeout names the same stage)
-enum F8Site { kF8Q = 0, kF8K = 1, kF8V = 2, kF8KVEmpty = 3, kF8S = 4, kF8P = 5, kF8O = 6, kF8Drain = 7 };
+enum F8Site { kF8Q = 0, kF8K = 1, kF8KVEmpty = 3, kF8S = 4, kF8P = 5, kF8O = 6, kF8Drain = 7 };
 
 struct F8Layout {
     static constexpr int kTileBytes = kTileM * kF8D;  // 128 rows x 128 e4m3
@@ -46,7 +46,7 @@ struct F8Layout {
     static constexpr int kK = kQ + 2 * kTileBytes;     // kF8Stages tiles
     static constexpr int kV = kK + kF8Stages * kTileBytes;
     static constexpr int kBar = kV + kF8Stages * kTileBytes;
-    static constexpr int kNumBars = 1 + 3 * kF8Stages + 3 * 2 + 1 + 1 + 2 * 2 + 2;  // ... unit ring, p_half0
+    static constexpr int kNumBars = 1 + 2 * kF8Stages + 3 * 2 + 1 + 1 + 2 * 2 + 2;  // ... unit ring, p_half0
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = kBytes + 1024;
@@ -172,10 +172,11 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
 
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
     uint64_t* q_full = bars + 0;
-    uint64_t* k_full = bars + 1;                 // [kF8Stages]
-    uint64_t* v_full = bars + 1 + kF8Stages;     // [kF8Stages]
-    uint64_t* kv_empty = bars + 1 + 2 * kF8Stages; // [kF8Stages]
-    uint64_t* s_full = bars + 1 + 3 * kF8Stages; // [2]
+    // [kF8Stages] K and V of a stage land on one barrier (one MMA-thread wait
+    // per key tile; a completed wait still idles the tensor core ~150 cycles)
+    uint64_t* k_full = bars + 1;
+    uint64_t* kv_empty = bars + 1 + kF8Stages;   // [kF8Stages]
+    uint64_t* s_full = bars + 1 + 2 * kF8Stages; // [2]
     uint64_t* p_full = s_full + 2;               // [2]
     uint64_t* o_full = p_full + 2;               // [2]
     uint64_t* drain = o_full + 2;
@@ -196,7 +197,6 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
         mbar_init(q_empty, 1);
         for (int s = 0; s < kF8Stages; ++s) {
             mbar_init(&k_full[s], 1);
-            mbar_init(&v_full[s], 1);
             mbar_init(&kv_empty[s], 1);
         }
         for (int s = 0; s < 2; ++s) {
@@ -257,10 +257,9 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     if (gk >= kF8Stages &&
                         !(ok = mbar_wait(&kv_empty[st], ((gk / kF8Stages) - 1) & 1, abort_flag, kF8KVEmpty)))
                         break;
-                    mbar_arrive_expect_tx(&k_full[st], L::kTileBytes);
+                    mbar_arrive_expect_tx(&k_full[st], 2 * L::kTileBytes);
                     tma_load_3d(smem + L::kK + st * L::kTileBytes, &tmK, &k_full[st], 0, j * kTileN, w.kvh);
-                    mbar_arrive_expect_tx(&v_full[st], L::kTileBytes);
-                    tma_load_3d(smem + L::kV + st * L::kTileBytes, &tmV, &v_full[st], 0, j * kTileN, w.kvh);
+                    tma_load_3d(smem + L::kV + st * L::kTileBytes, &tmV, &k_full[st], 0, j * kTileN, w.kvh);
                     n_kv = gk + 1;
                 }
                 if (!ok) break;
@@ -272,7 +271,6 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
             if (n_q > 0) f8_wait_drain(q_full, (n_q - 1) & 1, kF8Drain);
             for (int k = (n_kv > kF8Stages ? n_kv - kF8Stages : 0); k < n_kv; ++k) {
                 f8_wait_drain(&k_full[k % kF8Stages], (k / kF8Stages) & 1, kF8Drain);
-                f8_wait_drain(&v_full[k % kF8Stages], (k / kF8Stages) & 1, kF8Drain);
             }
         }
     } else if (warp == 8) {
@@ -333,15 +331,17 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                 for (int j = 0; j < n_iter; ++j) {
                     const int G = gk + j;
                     const int st = G % kF8Stages;
-                    const uint32_t ph = (G / kF8Stages) & 1;
                     const int sn = (G + 1) % kF8Stages;
                     const uint32_t sn_ph = ((G + 1) / kF8Stages) & 1;
-                    if (!(ok = mbar_wait(&v_full[st], ph, abort_flag, kF8V))) break;
+                    // V(G) arrived with K(G), waited for before S(j); the next
+                    // tile's barrier is waited for once, before the first S(j+1)
+                    bool next_kv = false;
                     if (j < nkv[0]) {
                         if (!(ok = issue_pv(0, st, j, (c0 + j) & 1))) break;
                         if (j == nkv[0] - 1) tc_commit(&o_full[0]);
                         if (j + 1 < nkv[0]) {
                             if (!(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
+                            next_kv = true;
                             tc_fence_after();
                             issue_s(0, sn);
                             tc_commit(&s_full[0]);
@@ -353,7 +353,7 @@ fa_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant
                     }
                     tc_commit(&kv_empty[st]);
                     if (j + 1 < nkv[1]) {
-                        if (!(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
+                        if (!next_kv && !(ok = mbar_wait(&k_full[sn], sn_ph, abort_flag, kF8K))) break;
                         tc_fence_after();
                         issue_s(1, sn);
                         tc_commit(&s_full[1]);
