@@ -34,7 +34,9 @@
 // scale*D x 2 stages | barriers.  Compute group g (query columns 64g ..
 // 64g+63) passes its 64 dQ rows through its 16 KB buffer as two 32-row
 // blocks; one thread of the group issues each bulk reduction and, before the
-// group refills the buffer, waits until the bulk engine has read it.  L2
+// group refills the buffer, waits until the bulk engine has read it.  The
+// group's four warps meet for this at two hardware named barriers per block
+// (an mbarrier round trip there cost ~200 cycles per hand-over).  L2
 // applies fp32 reductions at about 6 TB/s on this part, so a tile's 64 KB of
 // dQ takes roughly as long to leave as the tile's MMAs take to run; the dS
 // phase between the two blocks hides the first block's read.
@@ -65,7 +67,7 @@ constexpr int kMaxDynSmem = 232448;
 static_assert(kCols == 64, "the dS^T tile holds one 64-column swizzle atom per compute group");
 
 // wait sites (bits of the device status word)
-enum FusedSite { kFSmem = 8, kFLoad = 9, kFEmpty = 10, kFMma = 11, kFComp = 12, kFStage = 13, kFDrain = 14 };
+enum FusedSite { kFSmem = 8, kFLoad = 9, kFEmpty = 10, kFMma = 11, kFComp = 12, kFDrain = 14 };
 
 struct FusedLayout {
     static constexpr int kTileBytes = kTileM * kD * 2;        // 32 KB bf16 tile
@@ -81,7 +83,7 @@ struct FusedLayout {
     static constexpr int kLse = kStage + kGroups * kStageBytes;   // 2 stages x 128 fp32
     static constexpr int kDvec = kLse + 2 * kTileN * 4;           // 2 stages x 128 fp32
     static constexpr int kBar = kDvec + 2 * kTileN * 4;
-    static constexpr int kNumBars = 25;
+    static constexpr int kNumBars = 21;
     static constexpr int kMisc = kBar + kNumBars * 8;
     static constexpr int kBytes = kMisc + 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
@@ -161,8 +163,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint64_t* drain = bars + 16;
     uint64_t* unit_full = bars + 17;   // [2]
     uint64_t* unit_empty = bars + 19;  // [2]
-    uint64_t* stage_full = bars + 21;  // [2] per group: its dQ rows are staged
-    uint64_t* stage_free = bars + 23;  // [2] per group: its earlier reductions have read their staging
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
@@ -181,8 +181,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_init(&q_empty[s], 1);
             mbar_init(&unit_full[s], 1);
             mbar_init(&unit_empty[s], kCompute + 1);
-            mbar_init(&stage_full[s], kGroupThreads);
-            mbar_init(&stage_free[s], 1);
         }
         mbar_init(do_full, 1);
         mbar_init(do_empty, 1);
@@ -382,6 +380,12 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
         const int c0 = wg * kCols;       // this group's query columns
         const bool leader = (wq == 0 && lane == 0);   // issues the group's bulk reductions
+        // The group's two named barriers (128 threads): bar_stage before it
+        // refills its staging buffer (also reducing the warps' wait results, so
+        // that the four warps leave together), bar_staged once its rows are in
+        // the buffer (warps 1-3 arrive, warp 0 waits and issues the reduction).
+        const int bar_stage = 1 + 2 * wg;
+        const int bar_staged = 2 + 2 * wg;
         const float c = p.scale_log2;
         const float sc = p.scale;
         uint8_t* ds_s = smem + L::kDS;
@@ -396,52 +400,64 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         uint32_t va[32], vb[32];
         auto read_dq = [&](int gd) -> bool {
             const bool w_ok = mbar_wait(dq_full, gd & 1, abort_flag, kFComp);
-            if (!__all_sync(0xffffffffu, w_ok)) return false;
             tc_fence_after();
             tmem_ld32(tmem + lane_off + kColDP + c0, va);
             tmem_ld32(tmem + lane_off + kColDP + c0 + 32, vb);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(dq_free);
-            return true;
+            return w_ok;
         };
         // One 32-row block of the group's dQ rows (query tile i of head bhq;
         // block h = rows c0 + 32h ..) -> the group's staging buffer -> bulk
-        // reduction into the fp32 accumulator.  The buffer is reused once the
-        // group's previous reduction has read it (stage_free); every tile
-        // completes stage_free and stage_full twice, for h = 0 and h = 1.
-        auto stage_dq = [&](const uint32_t (&v)[32], int h, int bhq, int i) -> bool {
-            if (leader) {
-                bulk_wait_read_all();
-                mbar_arrive(&stage_free[wg]);
-            }
-            const bool w_ok = mbar_wait(&stage_free[wg], h, abort_flag, kFStage);
-            if (!__all_sync(0xffffffffu, w_ok)) return false;
+        // reduction into the fp32 accumulator.  The buffer is refilled once the
+        // leader's previous reduction has read it.  Every warp of the group
+        // calls this at the same points; it returns the AND over the group of
+        // the callers' `ok` (false: nothing staged, the group stops).
+        auto stage_dq = [&](const uint32_t (&v)[32], int h, int bhq, int i, bool ok) -> bool {
+            if (leader) bulk_wait_read_all();
+            __syncwarp();
+            if (!named_sync_and(bar_stage, kGroupThreads, ok)) return false;
 #pragma unroll
             for (int t = 0; t < 32; ++t) stage0[t * kD + r] = __uint_as_float(v[t]);
             fence_proxy_async_smem();
-            mbar_arrive(&stage_full[wg]);
-            if (leader && mbar_wait(&stage_full[wg], h, abort_flag, kFStage)) {
-                const int q0 = i * kTileM + c0 + h * L::kStageRows;
-                const int rows = max(0, min(L::kStageRows, p.N - q0));
-                if (rows > 0)
-                    bulk_reduce_add_f32(dq_sum + (static_cast<size_t>(bhq) * p.N + q0) * kD, stage0,
-                                        static_cast<uint32_t>(rows * kD * 4));
-                bulk_commit_group();
+            if (wq == 0) {
+                named_sync(bar_staged, kGroupThreads);
+                if (lane == 0) {
+                    const int q0 = i * kTileM + c0 + h * L::kStageRows;
+                    const int rows = max(0, min(L::kStageRows, p.N - q0));
+                    if (rows > 0)
+                        bulk_reduce_add_f32(dq_sum + (static_cast<size_t>(bhq) * p.N + q0) * kD, stage0,
+                                            static_cast<uint32_t>(rows * kD * 4));
+                    bulk_commit_group();
+                }
+                __syncwarp();
+            } else {
+                named_arrive(bar_staged, kGroupThreads);
             }
             return true;
         };
 
+        // ok: this thread's waits so far.  A failed wait (time limit, or
+        // another thread's abort) returns at once from then on; the thread
+        // goes on through the same steps on whatever the buffers hold (every
+        // address stays in bounds), keeping to the group's barrier sequence,
+        // and the group leaves together at its next bar_stage.
         bool ok = true;
         int g = 0;
-        for (int ui = 0; ok; ++ui) {
-            const int u = take_unit(ui, ok);
-            if (!__all_sync(0xffffffffu, ok) || u < 0) { ok = ok && u < 0; break; }
+        for (int ui = 0;; ++ui) {
+            bool u_ok;
+            const int u = take_unit(ui, u_ok);
+            ok = ok && u_ok;
+            __syncwarp();
+            if (!named_sync_and(bar_stage, kGroupThreads, ok)) { ok = false; break; }
+            if (u < 0) break;
             const FusedUnit w = fused_unit(p, T, u);
             const int j = w.j;
             const int kv = j * kTileN + r;
             const bool kv_ok = kv < p.N;
             const bool kv_block_partial = (j + 1) * kTileN > p.N;
+            bool left = false;   // the group stopped inside the unit
             for (int it = 0; it < w.n_it; ++it) {
                 const int gi = g + it;
                 const int st = gi & 1;
@@ -451,11 +467,10 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
                 const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
                 // ---- P^T = 2^(S^T c - lse2), handed to the dV MMAs in two halves
-                ok = mbar_wait(&q_full[st], (gi >> 1) & 1, abort_flag, kFComp) &&
-                     mbar_wait(s_full, ph, abort_flag, kFComp);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                tc_fence_after();
+                ok = mbar_wait(&q_full[st], (gi >> 1) & 1, abort_flag, kFComp) && ok;
+                ok = mbar_wait(s_full, ph, abort_flag, kFComp) && ok;
                 {
+                    tc_fence_after();
                     uint32_t sr[kCols / 32][32];
 #pragma unroll
                     for (int h = 0; h < kCols / 32; ++h) tmem_ld32(tmem + lane_off + kColS + c0 + h * 32, sr[h]);
@@ -496,91 +511,90 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 const int bhp = w.b * p.Hq + w.hkv * G + ghp;
                 const int ip = w.i0 + (it - 1 - ghp * w.per_head);
                 if (it > 0) {
-                    ok = read_dq(gi - 1) && stage_dq(va, 0, bhp, ip);
-                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                    ok = read_dq(gi - 1) && ok;
+                    if (!stage_dq(va, 0, bhp, ip, ok)) { left = true; break; }
                 }
                 // ---- dS^T = P^T o (dP^T - D) * scale -> shared memory (K-major, 128-byte swizzle)
-                ok = mbar_wait(dp_full, ph, abort_flag, kFComp);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                tc_fence_after();
+                ok = mbar_wait(dp_full, ph, abort_flag, kFComp) && ok;
+                {
+                    tc_fence_after();
 #pragma unroll
-                for (int h = 0; h < kCols / 32; ++h) {
-                    uint32_t dpr[32];
-                    tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
-                    tmem_ld_wait();
-                    uint32_t wv[16];
-                    const float2 sc2 = make_float2(sc, sc);
+                    for (int h = 0; h < kCols / 32; ++h) {
+                        uint32_t dpr[32];
+                        tmem_ld32(tmem + lane_off + kColDP + c0 + h * 32, dpr);
+                        tmem_ld_wait();
+                        uint32_t wv[16];
+                        const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) {
-                        // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
-                        const int q0 = h * 32 + 2 * t;
-                        const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
-                        const float2 gd = __ffma2_rn(
-                            make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2,
-                            make_float2(-dv2.x, -dv2.y));
-                        const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
-                        wv[t] = pack_bf16x2(d.x, d.y);
+                        for (int t = 0; t < 16; ++t) {
+                            // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
+                            const int q0 = h * 32 + 2 * t;
+                            const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
+                            const float2 gd = __ffma2_rn(
+                                make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2,
+                                make_float2(-dv2.x, -dv2.y));
+                            const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
+                            wv[t] = pack_bf16x2(d.x, d.y);
+                        }
+#pragma unroll
+                        for (int v = 0; v < 4; ++v) {
+                            const uint32_t off = sw128_offset(r, c0 + h * 32 + v * 8, kTileN);
+                            *reinterpret_cast<uint4*>(ds_s + off) =
+                                make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+                        }
                     }
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        const uint32_t off = sw128_offset(r, c0 + h * 32 + v * 8, kTileN);
-                        *reinterpret_cast<uint4*>(ds_s + off) =
-                            make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
-                    }
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(ds_full);
                 }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(ds_full);
-                if (it > 0) {
-                    ok = stage_dq(vb, 1, bhp, ip);
-                    if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-                }
+                if (it > 0 && !stage_dq(vb, 1, bhp, ip, ok)) { left = true; break; }
             }
-            if (!ok) break;
+            if (left) { ok = false; break; }
             // ---- the unit's last dQ^T
             {
                 const int itl = w.n_it - 1;
                 const int ghl = itl / w.per_head;
                 const int bhl = w.b * p.Hq + w.hkv * G + ghl;
                 const int il = w.i0 + (itl - ghl * w.per_head);
-                ok = read_dq(g + itl) && stage_dq(va, 0, bhl, il) && stage_dq(vb, 1, bhl, il);
-                if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+                ok = read_dq(g + itl) && ok;
+                if (!stage_dq(va, 0, bhl, il, ok) || !stage_dq(vb, 1, bhl, il, true)) { ok = false; break; }
             }
             // ---- epilogue: dV, dK rows of this key block (summed over the group)
-            ok = mbar_wait(dkv_full, ui & 1, abort_flag, kFComp);
-            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            tc_fence_after();
-            const size_t row = static_cast<size_t>(w.bkv) * p.N + kv;
-            constexpr int kPer = kD / kGroups;   // head-dimension columns written by this group
+            ok = mbar_wait(dkv_full, ui & 1, abort_flag, kFComp) && ok;
+            {
+                tc_fence_after();
+                const size_t row = static_cast<size_t>(w.bkv) * p.N + kv;
+                constexpr int kPer = kD / kGroups;   // head-dimension columns written by this group
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
-                __nv_bfloat16* dst_row =
-                    reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * kD + wg * kPer;
-                float* acc_row = p.a_dk ? (which == 0 ? p.a_dv : p.a_dk) + row * kD + wg * kPer : nullptr;
+                for (int which = 0; which < 2; ++which) {
+                    const uint32_t col0 = (which == 0 ? kColDV : kColDK) + wg * kPer;
+                    __nv_bfloat16* dst_row =
+                        reinterpret_cast<__nv_bfloat16*>(which == 0 ? p.dv : p.dk) + row * kD + wg * kPer;
+                    float* acc_row = p.a_dk ? (which == 0 ? p.a_dv : p.a_dk) + row * kD + wg * kPer : nullptr;
 #pragma unroll 1
-                for (int q = 0; q < kPer / 16; ++q) {
-                    uint32_t v16[16];
-                    tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
-                    tmem_ld_wait();
-                    if (acc_row) {   // accumulate mode: fp32 sums instead of bf16 outputs
-                        if (kv_ok) accumulate16(acc_row + q * 16, v16, p.a_first_dkv);
-                        continue;
-                    }
-                    uint32_t pk[8];
+                    for (int q = 0; q < kPer / 16; ++q) {
+                        uint32_t v16[16];
+                        tmem_ld16(tmem + lane_off + col0 + q * 16, v16);
+                        tmem_ld_wait();
+                        if (acc_row) {   // accumulate mode: fp32 sums instead of bf16 outputs
+                            if (kv_ok) accumulate16(acc_row + q * 16, v16, p.a_first_dkv);
+                            continue;
+                        }
+                        uint32_t pk[8];
 #pragma unroll
-                    for (int t = 0; t < 8; ++t)
-                        pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
-                    if (kv_ok) {
-                        uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
-                        dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-                        dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        for (int t = 0; t < 8; ++t)
+                            pk[t] = pack_bf16x2(__uint_as_float(v16[2 * t]), __uint_as_float(v16[2 * t + 1]));
+                        if (kv_ok) {
+                            uint4* dst = reinterpret_cast<uint4*>(dst_row + q * 16);
+                            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+                        }
                     }
                 }
+                // the next unit's dV / dK MMAs overwrite these columns only after this
+                // group's next P^T arrival (p_full0), which follows these completed loads
+                tc_fence_before();
             }
-            // the next unit's dV / dK MMAs overwrite these columns only after this
-            // group's next P^T arrival (p_full0), which follows these completed loads
-            tc_fence_before();
             g += w.n_it;
         }
         // the bulk engine must be done with shared memory before the CTA leaves
