@@ -458,12 +458,13 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             const bool kv_ok = kv < p.N;
             const bool kv_block_partial = (j + 1) * kTileN > p.N;
             bool left = false;   // the group stopped inside the unit
+            // query tile and head of the current and the previous iteration
+            int i = w.i0, bhq = w.b * p.Hq + w.hkv * G;
+            int ip = i, bhp = bhq;
             for (int it = 0; it < w.n_it; ++it) {
                 const int gi = g + it;
                 const int st = gi & 1;
                 const uint32_t ph = gi & 1;
-                const int gh = it / w.per_head;
-                const int i = w.i0 + (it - gh * w.per_head);
                 const float* lse_s = reinterpret_cast<const float*>(smem + L::kLse + st * kTileM * 4) + c0;
                 const float* dvec_s = reinterpret_cast<const float*>(smem + L::kDvec + st * kTileM * 4) + c0;
                 // ---- P^T = 2^(S^T c - lse2), handed to the dV MMAs in two halves
@@ -485,12 +486,15 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     const float2 c2 = make_float2(c, c);
                     static_for<0, 2>([&](auto hh) {
                         constexpr int h = decltype(hh)::value;
-                        static_for<0, 16>([&](auto tc) {
-                            constexpr int q = 32 * h + 2 * decltype(tc)::value;
-                            const float2 l2 = *reinterpret_cast<const float2*>(lse_s + q);
-                            const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l2.x, -l2.y));
+                        static_for<0, 8>([&](auto tc) {
+                            constexpr int q = 32 * h + 4 * decltype(tc)::value;
+                            const float4 l4 = *reinterpret_cast<const float4*>(lse_s + q);
+                            const float2 x = __ffma2_rn(make_float2(sv[q], sv[q + 1]), c2, make_float2(-l4.x, -l4.y));
+                            const float2 y = __ffma2_rn(make_float2(sv[q + 2], sv[q + 3]), c2, make_float2(-l4.z, -l4.w));
                             pv[q] = ex2(x.x);
                             pv[q + 1] = ex2(x.y);
+                            pv[q + 2] = ex2(y.x);
+                            pv[q + 3] = ex2(y.y);
                         });
                         if (masked) {
 #pragma unroll
@@ -507,9 +511,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 }
                 // ---- the previous query tile's dQ^T leaves tensor memory; its
                 //      first row block is reduced now, the second after dS
-                const int ghp = (it - 1) / w.per_head;
-                const int bhp = w.b * p.Hq + w.hkv * G + ghp;
-                const int ip = w.i0 + (it - 1 - ghp * w.per_head);
                 if (it > 0) {
                     ok = read_dq(gi - 1) && ok;
                     if (!stage_dq(va, 0, bhp, ip, ok)) { left = true; break; }
@@ -526,15 +527,20 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                         uint32_t wv[16];
                         const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-                        for (int t = 0; t < 16; ++t) {
+                        for (int t = 0; t < 16; t += 2) {
                             // dS = P (dP - D) scale = P fma(dP, scale, -scale*D); dvec holds scale*D
                             const int q0 = h * 32 + 2 * t;
-                            const float2 dv2 = *reinterpret_cast<const float2*>(dvec_s + q0);
-                            const float2 gd = __ffma2_rn(
+                            const float4 dv4 = *reinterpret_cast<const float4*>(dvec_s + q0);
+                            const float2 gd0 = __ffma2_rn(
                                 make_float2(__uint_as_float(dpr[2 * t]), __uint_as_float(dpr[2 * t + 1])), sc2,
-                                make_float2(-dv2.x, -dv2.y));
-                            const float2 d = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd);
-                            wv[t] = pack_bf16x2(d.x, d.y);
+                                make_float2(-dv4.x, -dv4.y));
+                            const float2 gd1 = __ffma2_rn(
+                                make_float2(__uint_as_float(dpr[2 * t + 2]), __uint_as_float(dpr[2 * t + 3])), sc2,
+                                make_float2(-dv4.z, -dv4.w));
+                            const float2 d0 = __fmul2_rn(make_float2(pv[q0], pv[q0 + 1]), gd0);
+                            const float2 d1 = __fmul2_rn(make_float2(pv[q0 + 2], pv[q0 + 3]), gd1);
+                            wv[t] = pack_bf16x2(d0.x, d0.y);
+                            wv[t + 1] = pack_bf16x2(d1.x, d1.y);
                         }
 #pragma unroll
                         for (int v = 0; v < 4; ++v) {
@@ -548,17 +554,17 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     mbar_arrive(ds_full);
                 }
                 if (it > 0 && !stage_dq(vb, 1, bhp, ip, ok)) { left = true; break; }
+                ip = i;
+                bhp = bhq;
+                if (++i == T) {
+                    i = w.i0;
+                    ++bhq;
+                }
             }
             if (left) { ok = false; break; }
-            // ---- the unit's last dQ^T
-            {
-                const int itl = w.n_it - 1;
-                const int ghl = itl / w.per_head;
-                const int bhl = w.b * p.Hq + w.hkv * G + ghl;
-                const int il = w.i0 + (itl - ghl * w.per_head);
-                ok = read_dq(g + itl) && ok;
-                if (!stage_dq(va, 0, bhl, il, ok) || !stage_dq(vb, 1, bhl, il, true)) { ok = false; break; }
-            }
+            // ---- the unit's last dQ^T (query tile ip of head bhp)
+            ok = read_dq(g + w.n_it - 1) && ok;
+            if (!stage_dq(va, 0, bhp, ip, ok) || !stage_dq(vb, 1, bhp, ip, true)) { ok = false; break; }
             // ---- epilogue: dV, dK rows of this key block (summed over the group)
             ok = mbar_wait(dkv_full, ui & 1, abort_flag, kFComp) && ok;
             {
