@@ -33,18 +33,20 @@
 // 128-byte swizzle) | dQ staging (fp32, 16 KB per compute group) | lse2,
 // scale*D x 2 stages | barriers.  Compute group g (query columns 64g ..
 // 64g+63) passes its 64 dQ rows through its 16 KB buffer as two 32-row
-// blocks; one thread of the group issues each bulk reduction and, before the
-// group refills the buffer, waits until the bulk engine has read it.  The
-// group's four warps meet for this at two hardware named barriers per block
-// (an mbarrier round trip there cost ~200 cycles per hand-over).  L2
+// blocks.  The group's threads wait until the buffer is free, store their
+// rows, and arrive on a barrier; a reduction warp of its own (one per group)
+// then issues the block's bulk reduction, waits until the bulk engine has
+// read the buffer and frees it.  The compute warps thus never wait for each
+// other or for the issue, only, before refilling, for the previous read.  L2
 // applies fp32 reductions at about 6 TB/s on this part, so a tile's 64 KB of
 // dQ takes roughly as long to leave as the tile's MMAs take to run; the dS
 // phase between the two blocks hides the first block's read.
 //
-// Warp roles (320 threads): warps 0-7 compute (thread = TMEM lane = key row
+// Warp roles (384 threads): warps 0-7 compute (thread = TMEM lane = key row
 // for P and dS, = head-dimension index for the dQ drain; warps 0-3 take query
 // columns 0-63, warps 4-7 columns 64-127), warp 8 issues MMAs (one thread),
-// warp 9 drives TMA.  Every wait is bounded (sm100.cuh).
+// warp 9 drives TMA, warps 10 and 11 issue the dQ reductions of compute
+// groups 0 and 1 (one thread each).  Every wait is bounded (sm100.cuh).
 #include "fa_internal.h"
 #include "sm100.cuh"
 
@@ -60,14 +62,15 @@ constexpr int kCols = kTileN / kGroups;     // query columns per compute group
 constexpr int kComputeWarps = 4 * kGroups;
 constexpr int kMmaWarp = kComputeWarps;
 constexpr int kLoadWarp = kComputeWarps + 1;
-constexpr int kThreads = 32 * (kComputeWarps + 2);
+constexpr int kReduceWarp = kComputeWarps + 2;   // + compute group: issues that group's dQ reductions
+constexpr int kThreads = 32 * (kComputeWarps + 2 + kGroups);
 constexpr int kCompute = 32 * kComputeWarps;
 constexpr int kGroupThreads = 128;
 constexpr int kMaxDynSmem = 232448;
 static_assert(kCols == 64, "the dS^T tile holds one 64-column swizzle atom per compute group");
 
 // wait sites (bits of the device status word)
-enum FusedSite { kFSmem = 8, kFLoad = 9, kFEmpty = 10, kFMma = 11, kFComp = 12, kFDrain = 14 };
+enum FusedSite { kFSmem = 8, kFLoad = 9, kFEmpty = 10, kFMma = 11, kFComp = 12, kFStage = 13, kFDrain = 14 };
 
 struct FusedLayout {
     static constexpr int kTileBytes = kTileM * kD * 2;        // 32 KB bf16 tile
@@ -83,9 +86,10 @@ struct FusedLayout {
     static constexpr int kLse = kStage + kGroups * kStageBytes;   // 2 stages x 128 fp32
     static constexpr int kDvec = kLse + 2 * kTileN * 4;           // 2 stages x 128 fp32
     static constexpr int kBar = kDvec + 2 * kTileN * 4;
-    static constexpr int kNumBars = 21;
+    static constexpr int kNumBars = 25;
     static constexpr int kMisc = kBar + kNumBars * 8;
-    static constexpr int kBytes = kMisc + 16;
+    static constexpr int kSlot = kMisc + 16;                  // [group][2] reduction target: offset, bytes
+    static constexpr int kBytes = kSlot + kGroups * 2 * 16;
     static constexpr int kAlloc = (kBytes + 1024 <= kMaxDynSmem) ? kBytes + 1024 : kMaxDynSmem;
     static_assert(kBytes <= kMaxDynSmem, "fused backward shared memory layout too large");
 };
@@ -163,6 +167,9 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
     uint64_t* drain = bars + 16;
     uint64_t* unit_full = bars + 17;   // [2]
     uint64_t* unit_empty = bars + 19;  // [2]
+    uint64_t* stage_full = bars + 21;  // [group]: the group's dQ rows are in its staging buffer
+    uint64_t* stage_free = bars + 23;  // [group]: the buffer's previous reduction has read it
+    unsigned long long* slot = reinterpret_cast<unsigned long long*>(smem + L::kSlot);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
     volatile int* unit_id = reinterpret_cast<volatile int*>(smem + L::kMisc + 8);  // [2]
@@ -180,7 +187,9 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
             mbar_init(&unit_full[s], 1);
-            mbar_init(&unit_empty[s], kCompute + 1);
+            mbar_init(&unit_empty[s], kCompute + 1 + kGroups);
+            mbar_init(&stage_full[s], kGroupThreads);
+            mbar_init(&stage_free[s], 1);
         }
         mbar_init(do_full, 1);
         mbar_init(do_empty, 1);
@@ -372,6 +381,35 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             tc_commit(drain);
             wait_drain(drain, 0, kFDrain);
         }
+    } else if (warp >= kReduceWarp) {
+        // ------------------------------------------------------------ dQ reductions of one group
+        // Round r of group c: wait until the group has staged its rows, issue
+        // the bulk reduction of the target the group's leader left in the slot,
+        // and release the buffer once the bulk engine has read it.  Two rounds
+        // per query tile (32 rows each), in the compute warps' unit order.
+        if (lane == 0) {
+            const int c = warp - kReduceWarp;
+            float* const dq_sum = p.a_dq ? p.a_dq : p.dq_acc;
+            const uint8_t* const buf = smem + L::kStage + c * L::kStageBytes;
+            bool ok = true;
+            int r = 0;
+            for (int ui = 0; ok; ++ui) {
+                const int u = take_unit(ui, ok);
+                if (!ok || u < 0) break;
+                const int rounds = 2 * fused_unit(p, T, u).n_it;
+                for (int k = 0; k < rounds; ++k, ++r) {
+                    if (!(ok = mbar_wait(&stage_full[c], r & 1, abort_flag, kFStage))) break;
+                    const unsigned long long* sl = slot + (c * 2 + (r & 1)) * 2;
+                    const unsigned long long off = sl[0], bytes = sl[1];
+                    if (bytes > 0) bulk_reduce_add_f32(dq_sum + off, buf, static_cast<uint32_t>(bytes));
+                    bulk_commit_group();
+                    bulk_wait_read_all();
+                    mbar_arrive(&stage_free[c]);
+                }
+            }
+            // the bulk engine must be done with shared memory before the CTA leaves
+            bulk_wait_all();
+        }
     } else {
         // ------------------------------------------------------------ compute (P^T, dQ drain, dS^T)
         const int wg = warp >> 2;
@@ -379,13 +417,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
         const int r = (wq << 5) + lane;  // TMEM lane: key row (P^T, dS^T) or head-dimension index (dQ^T)
         const uint32_t lane_off = static_cast<uint32_t>(wq << 5) << 16;
         const int c0 = wg * kCols;       // this group's query columns
-        const bool leader = (wq == 0 && lane == 0);   // issues the group's bulk reductions
-        // The group's two named barriers (128 threads): bar_stage before it
-        // refills its staging buffer (also reducing the warps' wait results, so
-        // that the four warps leave together), bar_staged once its rows are in
-        // the buffer (warps 1-3 arrive, warp 0 waits and issues the reduction).
-        const int bar_stage = 1 + 2 * wg;
-        const int bar_staged = 2 + 2 * wg;
+        const bool leader = (wq == 0 && lane == 0);   // names each block's reduction target
         const float c = p.scale_log2;
         const float sc = p.scale;
         uint8_t* ds_s = smem + L::kDS;
@@ -409,55 +441,44 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             return w_ok;
         };
         // One 32-row block of the group's dQ rows (query tile i of head bhq;
-        // block h = rows c0 + 32h ..) -> the group's staging buffer -> bulk
-        // reduction into the fp32 accumulator.  The buffer is refilled once the
-        // leader's previous reduction has read it.  Every warp of the group
-        // calls this at the same points; it returns the AND over the group of
-        // the callers' `ok` (false: nothing staged, the group stops).
-        auto stage_dq = [&](const uint32_t (&v)[32], int h, int bhq, int i, bool ok) -> bool {
-            if (leader) bulk_wait_read_all();
-            __syncwarp();
-            if (!named_sync_and(bar_stage, kGroupThreads, ok)) return false;
+        // block h = rows c0 + 32h ..) -> the group's staging buffer, once the
+        // group's reduction warp has seen the buffer's previous contents read
+        // by the bulk engine; that warp then reduces it into the fp32 sum.
+        int n_staged = 0;   // rounds of this group so far
+        auto stage_dq = [&](const uint32_t (&v)[32], int h, int bhq, int i, bool ok_in) -> bool {
+            bool w_ok = ok_in;
+            if (n_staged > 0) w_ok = mbar_wait(&stage_free[wg], (n_staged - 1) & 1, abort_flag, kFStage) && w_ok;
 #pragma unroll
             for (int t = 0; t < 32; ++t) stage0[t * kD + r] = __uint_as_float(v[t]);
-            fence_proxy_async_smem();
-            if (wq == 0) {
-                named_sync(bar_staged, kGroupThreads);
-                if (lane == 0) {
-                    const int q0 = i * kTileM + c0 + h * L::kStageRows;
-                    const int rows = max(0, min(L::kStageRows, p.N - q0));
-                    if (rows > 0)
-                        bulk_reduce_add_f32(dq_sum + (static_cast<size_t>(bhq) * p.N + q0) * kD, stage0,
-                                            static_cast<uint32_t>(rows * kD * 4));
-                    bulk_commit_group();
-                }
-                __syncwarp();
-            } else {
-                named_arrive(bar_staged, kGroupThreads);
+            if (leader) {
+                const int q0 = i * kTileM + c0 + h * L::kStageRows;
+                const int rows = max(0, min(L::kStageRows, p.N - q0));
+                unsigned long long* sl = slot + (wg * 2 + (n_staged & 1)) * 2;
+                sl[0] = (static_cast<unsigned long long>(bhq) * p.N + q0) * kD;
+                sl[1] = static_cast<unsigned long long>(rows) * kD * 4;
             }
-            return true;
+            fence_proxy_async_smem();
+            mbar_arrive(&stage_full[wg]);
+            ++n_staged;
+            return w_ok;
         };
 
         // ok: this thread's waits so far.  A failed wait (time limit, or
         // another thread's abort) returns at once from then on; the thread
-        // goes on through the same steps on whatever the buffers hold (every
-        // address stays in bounds), keeping to the group's barrier sequence,
-        // and the group leaves together at its next bar_stage.
+        // finishes the unit on whatever the buffers hold (every address stays
+        // in bounds) and leaves before the next one.
         bool ok = true;
         int g = 0;
         for (int ui = 0;; ++ui) {
             bool u_ok;
             const int u = take_unit(ui, u_ok);
-            ok = ok && u_ok;
-            __syncwarp();
-            if (!named_sync_and(bar_stage, kGroupThreads, ok)) { ok = false; break; }
-            if (u < 0) break;
+            ok = __all_sync(0xffffffffu, ok && u_ok);
+            if (!ok || u < 0) break;
             const FusedUnit w = fused_unit(p, T, u);
             const int j = w.j;
             const int kv = j * kTileN + r;
             const bool kv_ok = kv < p.N;
             const bool kv_block_partial = (j + 1) * kTileN > p.N;
-            bool left = false;   // the group stopped inside the unit
             // query tile and head of the current and the previous iteration
             int i = w.i0, bhq = w.b * p.Hq + w.hkv * G;
             int ip = i, bhp = bhq;
@@ -513,7 +534,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                 //      first row block is reduced now, the second after dS
                 if (it > 0) {
                     ok = read_dq(gi - 1) && ok;
-                    if (!stage_dq(va, 0, bhp, ip, ok)) { left = true; break; }
+                    ok = stage_dq(va, 0, bhp, ip, ok);
                 }
                 // ---- dS^T = P^T o (dP^T - D) * scale -> shared memory (K-major, 128-byte swizzle)
                 ok = mbar_wait(dp_full, ph, abort_flag, kFComp) && ok;
@@ -553,7 +574,7 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     tc_fence_before();
                     mbar_arrive(ds_full);
                 }
-                if (it > 0 && !stage_dq(vb, 1, bhp, ip, ok)) { left = true; break; }
+                if (it > 0) ok = stage_dq(vb, 1, bhp, ip, ok);
                 ip = i;
                 bhp = bhq;
                 if (++i == T) {
@@ -561,10 +582,10 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
                     ++bhq;
                 }
             }
-            if (left) { ok = false; break; }
             // ---- the unit's last dQ^T (query tile ip of head bhp)
             ok = read_dq(g + w.n_it - 1) && ok;
-            if (!stage_dq(va, 0, bhp, ip, ok) || !stage_dq(vb, 1, bhp, ip, true)) { ok = false; break; }
+            ok = stage_dq(va, 0, bhp, ip, ok);
+            ok = stage_dq(vb, 1, bhp, ip, ok);
             // ---- epilogue: dV, dK rows of this key block (summed over the group)
             ok = mbar_wait(dkv_full, ui & 1, abort_flag, kFComp) && ok;
             {
@@ -603,8 +624,6 @@ fa_bwd_fused_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_consta
             }
             g += w.n_it;
         }
-        // the bulk engine must be done with shared memory before the CTA leaves
-        if (leader) bulk_wait_all();
     }
 
     tc_fence_before();
