@@ -126,31 +126,6 @@ __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bu
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // ----------------------------------------------------------------------------
-// Named barriers (bar.sync / bar.arrive over `count` threads, a multiple of
-// 32; every warp that takes part executes the instruction with all its lanes).
-// A barrier completes once `count` threads have arrived; callers keep every
-// participating warp on the same sequence of barriers, so none waits for a
-// warp that has left.
-// ----------------------------------------------------------------------------
-__device__ __forceinline__ void named_sync(int id, int count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-__device__ __forceinline__ void named_arrive(int id, int count) {
-    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-// bar.sync that also returns the AND of the participating threads' predicates
-__device__ __forceinline__ bool named_sync_and(int id, int count, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\t"
-        "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, %2, %3, p;\n\t"
-        "selp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r) : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count) : "memory");
-    return r != 0;
-}
-
-// ----------------------------------------------------------------------------
 // tcgen05: tensor memory
 // ----------------------------------------------------------------------------
 // Whole warp: allocate `ncols` TMEM columns, address written to *slot (smem).
