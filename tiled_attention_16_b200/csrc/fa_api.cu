@@ -106,7 +106,9 @@ int sm_count() {
 namespace {
 
 // Split-KV plan of fa_decode: 64-key tiles, query rows in blocks of 16 per
-// K/V head, and enough key ranges that ~4 CTAs per SM stream the cache.
+// K/V head, and the number of key ranges that fills the resident CTA slots
+// (2 per SM at D = 128, 4 at D = 64: shared memory and registers) most
+// evenly over about two waves, so that no nearly empty last wave streams alone.
 struct DecodePlan {
     int n_row_blocks, n_splits, tiles_per_split;
     size_t o_part_off, lse_part_off, total;
@@ -131,9 +133,22 @@ DecodePlan decode_plan(const fa_kv_shape& s) {
     pl.n_row_blocks = (R + 15) / 16;
     const int n_tiles = (s.Nk + 63) / 64;
     const long long pairs = static_cast<long long>(s.B) * s.Hkv * pl.n_row_blocks;
-    const long long target = 4LL * 148;
-    long long splits = (target + pairs - 1) / pairs;
-    if (splits > n_tiles) splits = n_tiles;
+    const long long slots = 148LL * (s.D == 128 ? 2 : 4);
+    const long long s0 = (2 * slots + pairs - 1) / pairs;   // about two waves
+    long long splits = 1;
+    double best = -1.0;
+    for (long long c = (s0 + 1) / 2; c <= 2 * s0; ++c) {
+        const long long cs = c > n_tiles ? n_tiles : c;
+        // the ranges actually formed from cs: whole tiles per range
+        const long long per = (n_tiles + cs - 1) / cs;
+        const long long n = (n_tiles + per - 1) / per;
+        const double waves = static_cast<double>(pairs * n) / static_cast<double>(slots);
+        const double fill = waves / std::ceil(waves);
+        if (fill > best + 1e-9) {
+            best = fill;
+            splits = n;
+        }
+    }
     if (splits > 65535) splits = 65535;
     if (splits < 1) splits = 1;
     pl.tiles_per_split = static_cast<int>((n_tiles + splits - 1) / splits);
