@@ -225,6 +225,33 @@ def test_decode_workspace_covers_partials():
         assert A.lib().fa_decode_workspace_bytes(ctypes.byref(s)) >= rows * (s.D + 1) * 4
 
 
+def test_decode_plan_fills_the_resident_slots():
+    # The key-range count is chosen so that the split kernel's CTAs fill its
+    # resident slots (2 per SM at D = 128, 4 at D = 64; 148 SMs) in nearly
+    # whole waves.  The workspace holds rows x ranges x (D + 1) fp32, so it
+    # reveals the range count.
+    def ranges(**kw):
+        s = _kv(**kw)
+        rows = s.B * s.Hq * s.Nq
+        up = lambda x: (x + 255) // 256 * 256
+        need = A.lib().fa_decode_workspace_bytes(ctypes.byref(s))
+        found = [n for n in range(1, 4096) if up(rows * n * s.D * 4) + up(rows * n * 4) == need]
+        assert found, kw
+        return s, found[0]
+    # a 32K-token cache, 64 query / 8 K/V heads, 8 sequences: 64 (sequence, K/V head)
+    # pairs x 9 ranges = 576 CTAs on 296 slots (the former 10 left a 48-CTA third wave)
+    s, n = ranges(B=8, Hq=64, Hkv=8, Nq=1, Nk=32768, D=128)
+    assert n == 9
+    for kw in (dict(B=2, Hq=64, Hkv=8, Nq=1, Nk=16384, D=128), dict(B=4, Hq=32, Hkv=8, Nq=1, Nk=8192, D=64),
+               dict(B=1, Hq=8, Hkv=8, Nq=1, Nk=65536, D=128)):
+        s, n = ranges(**kw)
+        pairs = s.B * s.Hkv * ((s.Hq // s.Hkv * s.Nq + 15) // 16)
+        slots = 148 * (2 if s.D == 128 else 4)
+        waves = pairs * n / slots
+        # whole 64-key tiles per range limit the choice (8192 keys: 32, 43 or 64 ranges)
+        assert waves / -(-waves // 1) > 0.85, (kw, n, waves)
+
+
 # ---- sequence-sharded attention helpers (fa_lse_merge, fa_accumulate)
 def _merge(rows=64, D=128, o_part=P, lse_part=P, o_acc=P, lse_acc=P, o_out=None, first=0):
     return A.lib().fa_lse_merge(rows, D, o_part, lse_part, o_acc, lse_acc, o_out, first, None)
